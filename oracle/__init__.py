@@ -1,0 +1,187 @@
+"""CPU oracle for exact Lloyd k-means -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` may import this package.  The CUDA library never calls it and it
+never calls the CUDA library: the two share no code.
+
+The arithmetic lives in ``fk_oracle.c`` (fp64, direct-difference distance,
+first-minimum argmin, per-cluster mean, empty cluster keeps its previous
+centroid), following the problem statement of "Flash-KMeans: Fast and
+Memory-Efficient Exact K-Means" (arXiv 2603.09229, abstract: assignment stage
+plus centroid-update stage, exact).  This module adds numpy marshalling, the
+rounding of centroids to the input dtype and the Lloyd loop.
+
+Readings taken where the pages are silent:
+  * ties go to the lowest centroid index;
+  * an empty cluster keeps its previous centroid;
+  * centroids are kept in fp32 between iterations (the library's master copy)
+    and rounded to the input dtype (round-to-nearest-even) for the next
+    assignment, so both sides assign against the same rounded values.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fk_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH, openmp: bool = True) -> str:
+    """Compile the C oracle into a shared library (gcc, -O2, OpenMP)."""
+    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", src, "-o", out, "-lm"]
+    if openmp:
+        cmd.insert(1, "-fopenmp")
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lp = ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_assign.argtypes = [dp, ctypes.c_int64, ctypes.c_int, dp, ctypes.c_int, ip, dp, dp]
+    lib.oracle_assign.restype = None
+    lib.oracle_update.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, dp, lp]
+    lib.oracle_update.restype = ctypes.c_int
+    lib.oracle_objective.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp]
+    lib.oracle_objective.restype = ctypes.c_double
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def load(path: str = _LIB_PATH):
+    """Load (building first if needed) an oracle library; returns the ctypes handle."""
+    global _lib
+    if path == _LIB_PATH and _lib is not None:
+        return _lib
+    if not os.path.exists(path) or (path == _LIB_PATH and
+                                    os.path.getmtime(path) < os.path.getmtime(_SRC)):
+        build(out=path)
+    lib = _bind(ctypes.CDLL(path))
+    if path == _LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _p(a, t):
+    return a.ctypes.data_as(ctypes.POINTER(t))
+
+
+def num_threads() -> int:
+    return load().oracle_num_threads()
+
+
+def assign(X, C, lib=None):
+    """Nearest centroid per row.  Returns (labels int32, mindist f64, second f64)."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    N, D = X.shape
+    K = C.shape[0]
+    assert C.shape[1] == D and K >= 1
+    labels = np.zeros(N, np.int32)
+    mind = np.zeros(N, np.float64)
+    second = np.zeros(N, np.float64)
+    if N:
+        lib.oracle_assign(_p(X, ctypes.c_double), N, D, _p(C, ctypes.c_double), K,
+                          _p(labels, ctypes.c_int32), _p(mind, ctypes.c_double),
+                          _p(second, ctypes.c_double))
+    return labels, mind, second
+
+
+def update(X, labels, K, C_prev, lib=None):
+    """Per-cluster mean (fp64); empty clusters keep C_prev.  Returns (C_out, counts)."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    C_prev = np.ascontiguousarray(C_prev, dtype=np.float64)
+    N, D = X.shape
+    out = np.zeros((K, D), np.float64)
+    counts = np.zeros(K, np.int64)
+    rc = lib.oracle_update(_p(X, ctypes.c_double), _p(labels, ctypes.c_int32), N, D, K,
+                           _p(C_prev, ctypes.c_double), _p(out, ctypes.c_double),
+                           _p(counts, ctypes.c_int64))
+    if rc != 0:
+        raise ValueError("oracle_update: label out of range" if rc == -1 else "oracle_update failed")
+    return out, counts
+
+
+def objective(X, labels, C, lib=None) -> float:
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    return lib.oracle_objective(_p(X, ctypes.c_double), _p(labels, ctypes.c_int32),
+                                X.shape[0], X.shape[1], _p(C, ctypes.c_double))
+
+
+# ---------------------------------------------------------------- rounding --
+def to_f32(a) -> np.ndarray:
+    """fp64 -> fp32, round to nearest even (the C cast numpy performs)."""
+    return np.asarray(a, dtype=np.float64).astype(np.float32)
+
+
+def bf16_bits_from_f32(a) -> np.ndarray:
+    """fp32 -> bfloat16 bit patterns, round to nearest even on the dropped 16 bits."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(np.asarray(a, dtype=np.float32))
+    r[nan] = 0x7FC0
+    return r
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_to(dtype: str, a) -> np.ndarray:
+    """Value of ``a`` stored in ``dtype`` ("f64", "f32", "f16", "bf16"), as fp64.
+
+    fp16/bf16 round from fp32 (the library keeps fp32 master centroids)."""
+    a = np.asarray(a, dtype=np.float64)
+    if dtype == "f64":
+        return a.copy()
+    f32 = to_f32(a)
+    if dtype == "f32":
+        return f32.astype(np.float64)
+    if dtype == "f16":
+        return f32.astype(np.float16).astype(np.float64)
+    if dtype == "bf16":
+        return bf16_bits_to_f64(bf16_bits_from_f32(f32))
+    raise ValueError(dtype)
+
+
+# ------------------------------------------------------------------ Lloyd --
+def lloyd_step(X, C_master, dtype: str, lib=None):
+    """One Lloyd iteration from fp32 (or fp64 when dtype == "f64") master centroids.
+
+    Assignment uses the master rounded to ``dtype``; the update's empty-cluster
+    rule keeps the master value.  Returns (C_next master, labels, mindist,
+    second, counts)."""
+    Cr = round_to(dtype, C_master)
+    labels, mind, second = assign(X, Cr, lib)
+    Cn, counts = update(X, labels, Cr.shape[0], np.asarray(C_master, np.float64), lib)
+    Cn = Cn if dtype == "f64" else to_f32(Cn).astype(np.float64)
+    return Cn, labels, mind, second, counts
+
+
+def lloyd(X, C0, iters: int, dtype: str, lib=None):
+    """``iters`` Lloyd iterations.  Returns dict with final C, last labels /
+    mindist / counts and the objective of every assignment (list of floats)."""
+    C = np.asarray(C0, dtype=np.float64)
+    if dtype != "f64":
+        C = to_f32(C).astype(np.float64)
+    hist = []
+    labels = mind = counts = None
+    for _ in range(iters):
+        C, labels, mind, _, counts = lloyd_step(X, C, dtype, lib)
+        hist.append(float(mind.sum()))
+    return {"C": C, "labels": labels, "mindist": mind, "counts": counts, "objective": hist}

@@ -1,0 +1,117 @@
+/*
+ * fk_oracle.c -- plain, slow, obviously correct CPU oracle for one exact Lloyd
+ * k-means iteration.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and
+ * the benchmark's CPU-baseline leg use it to check and time the CUDA library;
+ * nothing in the product path links it, and it shares no code with it.
+ *
+ * What it computes follows "Flash-KMeans: Fast and Memory-Efficient Exact
+ * K-Means" (arXiv 2603.09229), abstract: the assignment stage gives each of N
+ * points its nearest of K centroids, the centroid-update stage replaces every
+ * centroid by the mean of the points assigned to it, and the method is exact,
+ * i.e. it reaches exactly this textbook Lloyd result.  Where the pages are
+ * silent the readings are: ties go to the lowest centroid index; a centroid
+ * that receives no point keeps its previous value.
+ *
+ * All arithmetic is fp64, points and centroids are row-major (N x D, K x D).
+ * The distance is the direct difference sum_j (x_j - c_j)^2, not the expanded
+ * |x|^2 + |c|^2 - 2<x,c> form the GPU uses.  Sums run in index order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads an OpenMP region of this library uses (1 without OpenMP). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Squared Euclidean distance, written out as the definition. */
+static double sqdist(const double *x, const double *c, int D) {
+    double s = 0.0;
+    for (int j = 0; j < D; ++j) {
+        double t = x[j] - c[j];
+        s += t * t;
+    }
+    return s;
+}
+
+/*
+ * Assignment stage: labels[i] = the first k (lowest index) reaching
+ * min_k |x_i - c_k|^2; mindist[i] = that minimum; second[i] (nullable) = the
+ * smallest distance over all other centroids (+inf when K == 1), which the
+ * parity tests use to recognise near-ties.
+ */
+void oracle_assign(const double *X, int64_t N, int D, const double *C, int K,
+                   int32_t *labels, double *mindist, double *second) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double *x = X + (size_t)i * (size_t)D;
+        double best = INFINITY, runner = INFINITY;
+        int32_t arg = 0;
+        for (int k = 0; k < K; ++k) {
+            double d = sqdist(x, C + (size_t)k * (size_t)D, D);
+            if (d < best) {
+                runner = best;
+                best = d;
+                arg = k;
+            } else if (d < runner) {
+                runner = d;
+            }
+        }
+        labels[i] = arg;
+        if (mindist) mindist[i] = best;
+        if (second) second[i] = runner;
+    }
+}
+
+/*
+ * Centroid-update stage: counts[k] = #{i : labels[i] == k};
+ * C_out[k] = (sum of those x_i) / counts[k], or C_prev[k] when counts[k] == 0.
+ * Returns 0, or -1 if a label lies outside [0, K).
+ */
+int oracle_update(const double *X, const int32_t *labels, int64_t N, int D, int K,
+                  const double *C_prev, double *C_out, int64_t *counts) {
+    double *sums = (double *)calloc((size_t)K * (size_t)D, sizeof(double));
+    if (!sums) return -2;
+    for (int k = 0; k < K; ++k) counts[k] = 0;
+    for (int64_t i = 0; i < N; ++i) {
+        int32_t k = labels[i];
+        if (k < 0 || k >= K) {
+            free(sums);
+            return -1;
+        }
+        counts[k] += 1;
+        const double *x = X + (size_t)i * (size_t)D;
+        double *s = sums + (size_t)k * (size_t)D;
+        for (int j = 0; j < D; ++j) s[j] += x[j];
+    }
+    for (int k = 0; k < K; ++k) {
+        double *out = C_out + (size_t)k * (size_t)D;
+        if (counts[k] > 0) {
+            const double *s = sums + (size_t)k * (size_t)D;
+            for (int j = 0; j < D; ++j) out[j] = s[j] / (double)counts[k];
+        } else {
+            const double *prev = C_prev + (size_t)k * (size_t)D;
+            for (int j = 0; j < D; ++j) out[j] = prev[j];
+        }
+    }
+    free(sums);
+    return 0;
+}
+
+/* Lloyd objective J = sum_i |x_i - c_{labels[i]}|^2. */
+double oracle_objective(const double *X, const int32_t *labels, int64_t N, int D,
+                        const double *C) {
+    double J = 0.0;
+    for (int64_t i = 0; i < N; ++i)
+        J += sqdist(X + (size_t)i * (size_t)D, C + (size_t)labels[i] * (size_t)D, D);
+    return J;
+}

@@ -1,0 +1,282 @@
+"""Pins for the CPU oracle (no GPU).
+
+The Flash-KMeans pages (arXiv 2603.09229 abstract; the Japanese HN summary,
+section on what Flash-KMeans changes) print no worked example, so the oracle is
+pinned to things other than itself:
+
+* library routines that solve a special case: ``scipy.cluster.vq.vq`` (nearest
+  code-book entry) and ``sklearn.cluster.KMeans`` limited to one Lloyd step;
+* closed forms and hand-worked cases (K = 1 gives the global mean; a 1-D
+  example; centroids equal to data rows);
+* invariants of Lloyd's algorithm (counts sum to N, each centroid is the mean
+  of its members, the objective never increases);
+* recovery of a planted, well-separated mixture;
+* the tie and empty-cluster readings (lowest index; keep previous centroid).
+
+``test_mutants_are_caught`` plants plausible mistakes in a copy of the C
+source and checks that the pins above reject every one of them.
+"""
+import os
+import re
+import tempfile
+
+import numpy as np
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+# ----------------------------------------------------------------- pins ----
+def pin_vq(lib):
+    from scipy.cluster.vq import vq
+    rng = np.random.default_rng(1)
+    for (N, D, K) in [(300, 3, 7), (257, 1, 5), (64, 33, 64), (50, 8, 1)]:
+        X = rng.standard_normal((N, D))
+        C = rng.standard_normal((K, D))
+        lab, mind, second = oracle.assign(X, C, lib)
+        code, dist = vq(X, C, check_finite=True)
+        assert np.array_equal(lab, code.astype(np.int32)), (N, D, K)
+        np.testing.assert_allclose(mind, dist ** 2, rtol=1e-9, atol=1e-12)
+        full = ((X[:, None, :] - C[None, :, :]) ** 2).sum(-1)
+        if K > 1:
+            full[np.arange(N), lab] = np.inf
+            np.testing.assert_allclose(second, full.min(1), rtol=1e-9, atol=1e-12)
+        else:
+            assert np.all(np.isinf(second))
+
+
+def pin_sklearn_step(lib):
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(2)
+    for (N, D, K) in [(500, 5, 7), (400, 16, 20)]:
+        X = rng.standard_normal((N, D)) + 3.0 * rng.integers(0, 4, (N, 1))
+        C0 = X[:K].copy()
+        lab, _, _ = oracle.assign(X, C0, lib)
+        Cn, counts = oracle.update(X, lab, K, C0, lib)
+        assert counts.min() > 0  # sklearn relocates empty clusters; avoid them here
+        km = KMeans(n_clusters=K, init=C0, n_init=1, max_iter=1, algorithm="lloyd",
+                    tol=0.0).fit(X)
+        np.testing.assert_allclose(Cn, km.cluster_centers_, rtol=1e-10, atol=1e-12)
+
+
+def pin_hand_1d(lib):
+    # points 0,1,9,10,4 against centroids 0 and 10 (worked by hand):
+    # squared distances (0,100) (1,81) (81,1) (100,0) (16,36)
+    X = np.array([[0.0], [1.0], [9.0], [10.0], [4.0]])
+    C = np.array([[0.0], [10.0]])
+    lab, mind, second = oracle.assign(X, C, lib)
+    assert lab.tolist() == [0, 0, 1, 1, 0]
+    assert mind.tolist() == [0.0, 1.0, 1.0, 0.0, 16.0]
+    assert second.tolist() == [100.0, 81.0, 81.0, 100.0, 36.0]
+    Cn, counts = oracle.update(X, lab, 2, C, lib)
+    assert counts.tolist() == [3, 2]
+    assert Cn[0, 0] == pytest.approx(5.0 / 3.0, abs=1e-15) and Cn[1, 0] == 9.5
+    # 2-D: x = (1, 2), c0 = (4, 6) -> 9 + 16 = 25, c1 = (1, -1) -> 0 + 9 = 9
+    lab, mind, _ = oracle.assign(np.array([[1.0, 2.0]]), np.array([[4.0, 6.0], [1.0, -1.0]]), lib)
+    assert lab.tolist() == [1] and mind.tolist() == [9.0]
+
+
+def pin_ties(lib):
+    # x = 5 is equidistant (25) from 0 and 10: the lower index wins, whatever the values
+    X = np.array([[5.0], [5.0]])
+    assert oracle.assign(X, np.array([[0.0], [10.0]]), lib)[0].tolist() == [0, 0]
+    assert oracle.assign(X, np.array([[10.0], [0.0]]), lib)[0].tolist() == [0, 0]
+    # duplicated centroids: the first copy wins
+    C = np.array([[9.0, 9.0], [1.0, 1.0], [1.0, 1.0], [1.0, 1.0]])
+    X = np.array([[1.0, 2.0], [0.0, 0.0], [9.0, 9.0]])
+    assert oracle.assign(X, C, lib)[0].tolist() == [1, 1, 0]
+    # small-integer lattice: ties exact in fp64, brute-force first minimum
+    rng = np.random.default_rng(3)
+    X = rng.integers(-3, 4, (200, 3)).astype(np.float64)
+    C = rng.integers(-3, 4, (9, 3)).astype(np.float64)
+    lab, mind, _ = oracle.assign(X, C, lib)
+    for i in range(len(X)):
+        d = [int(((X[i] - C[k]) ** 2).sum()) for k in range(len(C))]
+        assert lab[i] == d.index(min(d)) and mind[i] == min(d)
+
+
+def pin_k1_mean(lib):
+    rng = np.random.default_rng(4)
+    X = rng.standard_normal((123, 6))
+    lab, mind, _ = oracle.assign(X, X[:1], lib)
+    assert np.all(lab == 0)
+    Cn, counts = oracle.update(X, lab, 1, X[:1], lib)
+    assert counts.tolist() == [123]
+    np.testing.assert_allclose(Cn[0], X.mean(0), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(mind, ((X - X[0]) ** 2).sum(1), rtol=1e-12, atol=1e-14)
+
+
+def pin_prefix_identity(lib):
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((90, 4))
+    K = 30
+    lab, mind, second = oracle.assign(X, X[:K], lib)
+    assert lab[:K].tolist() == list(range(K))
+    assert np.all(mind[:K] == 0.0) and np.all(second[:K] > 0)
+
+
+def pin_permutation(lib):
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal((400, 5))
+    C = rng.standard_normal((13, 5))
+    perm = rng.permutation(13)
+    l1, m1, _ = oracle.assign(X, C, lib)
+    l2, m2, _ = oracle.assign(X, C[perm], lib)
+    # centroid perm[j] sits at position j, so label l1 -> position inv[l1]
+    inv = np.argsort(perm)
+    assert np.array_equal(l2, inv[l1]) and np.array_equal(m1, m2)
+
+
+def pin_empty_cluster(lib):
+    X = np.array([[0.0, 0.0], [0.1, 0.0], [5.0, 5.0]])
+    C = np.array([[0.0, 0.0], [100.0, 100.0], [5.0, 5.0]])
+    lab, _, _ = oracle.assign(X, C, lib)
+    assert lab.tolist() == [0, 0, 2]
+    Cn, counts = oracle.update(X, lab, 3, C, lib)
+    assert counts.tolist() == [2, 0, 1]
+    assert Cn[1].tolist() == [100.0, 100.0]
+    np.testing.assert_allclose(Cn[0], [0.05, 0.0], rtol=0, atol=1e-15)
+
+
+def pin_invariants(lib):
+    rng = np.random.default_rng(7)
+    N, D, K = 600, 4, 9
+    X = rng.standard_normal((N, D)) + 4.0 * rng.integers(0, 3, (N, D))
+    out = None
+    C = X[:K].copy()
+    J_prev = np.inf
+    for _ in range(8):
+        lab, mind, _ = oracle.assign(X, C, lib)
+        J = mind.sum()
+        assert J <= J_prev * (1 + 1e-12)
+        Cn, counts = oracle.update(X, lab, K, C, lib)
+        assert counts.sum() == N
+        sums = np.zeros((K, D))
+        np.add.at(sums, lab, X)
+        nz = counts > 0
+        np.testing.assert_allclose(Cn[nz], sums[nz] / counts[nz, None], rtol=1e-12, atol=1e-13)
+        # the update never increases the objective for fixed labels
+        assert oracle.objective(X, lab, Cn, lib) <= J * (1 + 1e-12)
+        J_prev, C = J, Cn
+    out = oracle.lloyd(X, X[:K], 8, "f64", lib)
+    h = out["objective"]
+    assert all(b <= a * (1 + 1e-12) for a, b in zip(h, h[1:]))
+
+
+def pin_planted(lib):
+    rng = np.random.default_rng(8)
+    K, D, per = 12, 6, 40
+    centers = rng.uniform(-50, 50, (K, D))
+    comp = np.repeat(np.arange(K), per)
+    X = centers[comp] + 0.01 * rng.standard_normal((K * per, D))
+    lab, _, _ = oracle.assign(X, centers, lib)
+    assert np.array_equal(lab, comp)
+    Cn, counts = oracle.update(X, lab, K, centers, lib)
+    assert counts.tolist() == [per] * K
+    for k in range(K):
+        np.testing.assert_allclose(Cn[k], X[comp == k].mean(0), rtol=1e-12, atol=1e-12)
+
+
+PINS = [pin_vq, pin_sklearn_step, pin_hand_1d, pin_ties, pin_k1_mean, pin_prefix_identity,
+        pin_permutation, pin_empty_cluster, pin_invariants, pin_planted]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_pin(pin, oracle_lib):
+    pin(oracle_lib)
+
+
+def test_update_rejects_bad_label(oracle_lib):
+    with pytest.raises(ValueError):
+        oracle.update(np.zeros((3, 2)), np.array([0, 2, 1], np.int32), 2, np.zeros((2, 2)), oracle_lib)
+
+
+# ------------------------------------------------------------- rounding ----
+def test_bf16_rounding_nearest_even():
+    import torch
+    one = 1.0
+    vals = np.array([one, one + 2 ** -8, one + 3 * 2 ** -8, -2.5, 3.0e38, 1e-40, 0.0, -0.0,
+                     np.inf, -np.inf], np.float32)
+    bits = oracle.bf16_bits_from_f32(vals)
+    assert bits[0] == 0x3F80 and bits[1] == 0x3F80 and bits[2] == 0x3F82
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(bits, ref)
+    rng = np.random.default_rng(9)
+    v = (rng.standard_normal(100000) * 10.0 ** rng.integers(-20, 20, 100000)).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(oracle.bf16_bits_from_f32(v), ref)
+
+
+def test_round_to_f16_matches_torch():
+    import torch
+    rng = np.random.default_rng(10)
+    v = rng.standard_normal(50000) * 100
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float16).double().numpy()
+    assert np.array_equal(oracle.round_to("f16", v), ref)
+
+
+def test_lloyd_loop_matches_manual_steps(oracle_lib):
+    rng = np.random.default_rng(11)
+    X = oracle.round_to("bf16", rng.standard_normal((300, 8)))
+    out = oracle.lloyd(X, X[:5], 3, "bf16", oracle_lib)
+    C = X[:5].copy()
+    for _ in range(3):
+        Cr = oracle.round_to("bf16", C)
+        lab, mind, _ = oracle.assign(X, Cr, oracle_lib)
+        Cn, _ = oracle.update(X, lab, 5, C, oracle_lib)
+        C = Cn.astype(np.float32).astype(np.float64)
+    assert np.array_equal(out["C"], C) and np.array_equal(out["labels"], lab)
+
+
+# ---------------------------------------------------------------- golden ---
+def test_golden_fixture(oracle_lib):
+    """Regression pin: values written by tests/golden/make_golden.py (oracle only)."""
+    import json
+    import workloads
+    path = os.path.join(HERE, "golden", "tiny_f32_n512_k16.json")
+    with open(path) as f:
+        g = json.load(f)
+    s = workloads.spec("tiny_f32", N=g["N"], K=g["K"], n_centers=g["n_centers"])
+    w = workloads.make(s, seed=g["seed"])
+    X = w.X.double().numpy()
+    out = oracle.lloyd(X, w.C0.double().numpy(), g["iters"], "f32", oracle_lib)
+    assert out["labels"].tolist() == g["labels"]
+    assert out["counts"].tolist() == g["counts"]
+    np.testing.assert_allclose(out["C"], np.array(g["C"]), rtol=0, atol=0)
+
+
+# --------------------------------------------------------------- mutants ---
+MUTANTS = [
+    ("wrong sign", "double t = x[j] - c[j];", "double t = x[j] + c[j];"),
+    ("no square", "s += t * t;", "s += fabs(t);"),
+    ("dropped accumulation", "s += t * t;", "s = t * t;"),
+    ("tie to highest index", "if (d < best) {", "if (d <= best) {"),
+    ("centroid stride", "sqdist(x, C + (size_t)k * (size_t)D, D)", "sqdist(x, C + (size_t)k, D)"),
+    ("runner-up not tracked", "runner = best;\n", "\n"),
+    ("mean off by one", "out[j] = s[j] / (double)counts[k];", "out[j] = s[j] / (double)(counts[k] + 1);"),
+    ("empty cluster zeroed", "for (int j = 0; j < D; ++j) out[j] = prev[j];",
+     "for (int j = 0; j < D; ++j) out[j] = 0.0;"),
+    ("last point dropped", "for (int64_t i = 0; i < N; ++i) {\n        int32_t k = labels[i];",
+     "for (int64_t i = 0; i + 1 < N; ++i) {\n        int32_t k = labels[i];"),
+]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=lambda m: m[0])
+def test_mutants_are_caught(mutant):
+    name, old, new = mutant
+    src = open(oracle._SRC).read()
+    assert src.count(old) >= 1, name
+    with tempfile.TemporaryDirectory() as td:
+        path = os.path.join(td, "mutant.c")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        lib = oracle._bind(__import__("ctypes").CDLL(oracle.build(path, os.path.join(td, "m.so"), openmp=False)))
+        caught = []
+        for pin in PINS:
+            try:
+                pin(lib)
+            except (AssertionError, ValueError):
+                caught.append(pin.__name__)
+        assert caught, f"mutant '{name}' passes every pin"
