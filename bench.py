@@ -1,0 +1,410 @@
+"""Benchmark: exact Lloyd k-means iterations per second on B200.
+
+One step = one pass of the whole hot path on the embedding workload
+(N = 1,048,576 points, D = 128, fp16, K = 1,024 centroids; the workload the
+headline metric is quoted on):
+
+    fk_prepare_centroids  (round fp32 centroids to fp16, centroid norms)
+    fk_assign_prepared    (tcgen05 FlashAssign: distances + online argmin)
+    fk_update             (sort-inverse update: radix sort, segment offsets,
+                           segmented sums, divide)
+
+all through the C ABI, inputs resident in HBM (X = 256 MiB, larger than the
+126 MB L2, so no flush is needed between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu]
+
+Prints one JSON line (rank 0).  Multi-GPU runs are replicas: every rank runs
+its own copy of the workload, there is no collective on the data path, the
+time is the max over ranks and the value is the sum of all ranks' steps
+divided by it ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "k-means Lloyd iter/s; assign TFLOP/s & update GB/s as % of B200 roofline"
+UNIT = "iter/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------- rank helpers --
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(steps_per_rank: int, elapsed_ms: float, world: int, device=None):
+    """Whole-job throughput: all ranks' steps over the slowest rank's time."""
+    t_max = max_over_ranks(elapsed_ms, world, device)
+    units = sum_over_ranks(float(steps_per_rank), world, device)
+    return units / (t_max / 1e3), t_max
+
+
+# ----------------------------------------------------------------- peaks --
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled in the background."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 20):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.period = period_ms
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", str(self.period)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self._t:
+                self._t.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        def parse(r):
+            f = [x.strip() for x in r.split(",")]
+            try:
+                return {"sm": float(f[1]), "max": float(f[2]), "active": f[4],
+                        "hw_slowdown": f[5], "hw_thermal_slowdown": f[6],
+                        "sw_thermal_slowdown": f[7], "sw_power_cap": f[8]}
+            except (ValueError, IndexError):
+                return None
+        inside = [parse(r) for (t, r) in self.rows if t0 <= t <= t1]
+        inside = [x for x in inside if x]
+        window = "timed"
+        if not inside:  # region shorter than the sampling period: nearest samples
+            near = sorted(self.rows, key=lambda tr: min(abs(tr[0] - t0), abs(tr[0] - t1)))[:3]
+            inside = [x for x in (parse(r) for _, r in near) if x]
+            window = "nearest to timed region"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        reasons = sorted({k for x in inside for k in ("hw_slowdown", "hw_thermal_slowdown",
+                                                       "sw_thermal_slowdown", "sw_power_cap")
+                          if x[k].lower() == "active"})
+        return {"sm_mhz": statistics.median(x["sm"] for x in inside),
+                "sm_max_mhz": max(x["max"] for x in inside), "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+# --------------------------------------------------------- profile data --
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("assign_tc.cu", "fk_common.cuh"):
+        with open(os.path.join(ROOT, "distance_argmin_flashassign_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the assign kernel from the committed ncu
+    summary, or None when absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"assign_tc_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        p = json.load(f)
+    if p.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return p.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_throughput(X64, C64, dtype: str, N_full: int, budget_s: float):
+    """Time the oracle's Lloyd step on a sample of rows (all K centroids) and
+    scale it linearly in N to iterations per second of the full workload."""
+    import numpy as np
+
+    import oracle
+    lib = oracle.load()
+    n = min(256, X64.shape[0])
+    t = time.perf_counter()
+    oracle.lloyd_step(X64[:n], C64, dtype, lib)
+    per_row = (time.perf_counter() - t) / n
+    n = int(max(256, min(X64.shape[0], budget_s / max(per_row, 1e-9))))
+    t = time.perf_counter()
+    oracle.lloyd_step(X64[:n], C64, dtype, lib)
+    dt = time.perf_counter() - t
+    value = n / (N_full * dt)
+    return value, n, dt, oracle.num_threads()
+
+
+# ------------------------------------------------------------- workloads --
+def build_inputs(name: str, device, seed: int):
+    import workloads
+    s = workloads.spec(name)
+    w = workloads.make(s, seed=seed, device=device)
+    return s, w
+
+
+def bench_gpu(args):
+    import torch
+
+    import distance_argmin_flashassign_b200 as fk
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    s, w = build_inputs(args.workload, dev, seed=rank)
+    dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[s.dtype]
+    X = w.X
+    B, N, D, K = s.B, s.N, s.D, s.K
+    C = w.C0.clone()
+    C_dt, norms = fk.fk_prepare_centroids(C, dt)
+    labels = torch.empty(((B, N) if B > 1 else (N,)), dtype=torch.int32, device=dev)
+    counts = torch.empty(((B, K) if B > 1 else (K,)), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        fk.fk_prepare_centroids(C, dt, C_dt, norms)
+        if ev:
+            ev[0].record(stream)
+        fk.fk_assign_prepared(X, C_dt, norms, labels)
+        if ev:
+            ev[1].record(stream)
+        fk.fk_update(X, labels, C, counts)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    fk.fk_sync()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start before the timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = fk.fk_launch_count()
+    w0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    launches = fk.fk_launch_count() - n0
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    fk.fk_sync()
+    elapsed = t_start.elapsed_time(t_end)
+    t_assign = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_update = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    value, t_max = aggregate(args.steps, elapsed, world, dev)
+    peaks, peak_kind = load_peaks()
+    flops = 2.0 * B * N * K * D
+    es = s.bytes_per_elem
+    upd_bytes = B * (N * D * es + 4 * N + K * (4 * D + 4))
+    tflops = flops / (t_assign * 1e-3) / 1e12
+    gbs = upd_bytes / (t_update * 1e-3) / 1e9
+    roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": round(tflops, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
+                "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
+                "traffic": profiled_traffic(args.workload), "ms_per_launch": round(t_assign, 5),
+                "algorithmic_flops_per_launch": flops}
+    roofline_update = {"bound": "hbm", "kernels": "fk_update (sort, offsets, segsum, finalize)",
+                       "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peak_kind} copy",
+                       "ms_per_call": round(t_update, 5), "algorithmic_bytes_per_call": upd_bytes}
+
+    out = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+           "config": {"workload": args.workload, "N": N, "D": D, "K": K, "B": B, "dtype": s.dtype,
+                      "step": "one Lloyd iteration: prepare centroids + assign + update",
+                      "l2": "inputs larger than L2 (X is %d MiB)" % (B * N * D * es >> 20),
+                      "parallelism": "replicas" if world > 1 else "single GPU"},
+           "roofline": roofline, "roofline_update": roofline_update,
+           "gpu_launches": launches,
+           "clocks": clocks.summary(w0, w1)}
+
+    if args.e2e:
+        out["e2e"] = bench_e2e(args, s, w, fk, dev, world)
+    if rank == 0 and world == 1 and args.cpu:
+        import workloads  # noqa: F401
+        X64 = X[: min(N, 65536)].double().cpu().numpy() if B == 1 else X[0, : min(N, 65536)].double().cpu().numpy()
+        C64 = w.C0.double().cpu().numpy() if B == 1 else w.C0[0].double().cpu().numpy()
+        v, n, secs, cores = oracle_throughput(X64, C64, s.dtype, N * B, args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{n} of {N * B} rows against all {K} centroids, one Lloyd step "
+                                         f"({secs:.1f} s), scaled linearly in N"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def bench_e2e(args, s, w, fk, dev, world):
+    """Same metric through fk_lloyd_ooc with host buffers: every step copies X
+    (pinned) to the device in chunks, runs one Lloyd iteration and copies the
+    labels, centroids and counts back."""
+    import torch
+    B, N, D, K = s.B, s.N, s.D, s.K
+    if B != 1:
+        return None
+    Xh = w.X.cpu().pin_memory()
+    Ch = w.C0.cpu().clone()
+    lab_h = torch.empty(N, dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty(K, dtype=torch.int32).pin_memory()
+    chunk = max(1, N // 4)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(min(args.warmup, 2)):
+        fk.fk_lloyd_ooc(Xh, Ch, 1, chunk, lab_h, cnt_h)
+    steps = max(1, min(args.steps, args.e2e_steps))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for _ in range(steps):
+        fk.fk_lloyd_ooc(Xh, Ch, 1, chunk, lab_h, cnt_h)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    value, _ = aggregate(steps, t0.elapsed_time(t1), world, dev)
+    es = s.bytes_per_elem
+    return {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": N * D * es + K * D * 4,
+            "d2h_bytes_per_step": N * 4 + K * D * 4 + K * 4, "steps": steps,
+            "api": "fk_lloyd_ooc(iters=1, chunk_rows=N/4), pinned host X"}
+
+
+# -------------------------------------------------------- reference arm --
+def bench_reference(args):
+    """The oracle, as it stands, on the host cores: each step is one Lloyd
+    step of the oracle on a bounded row sample of the same workload, scaled
+    linearly in N.  Only rank 0 works and prints under torchrun."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    import workloads
+    s = workloads.spec(args.workload)
+    per_step = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
+    w = workloads.make(s.replace(B=1) if s.B > 1 else s, seed=0, device="cpu")
+    X64 = w.X[: min(s.N, 65536)].double().numpy()
+    C64 = w.C0.double().numpy()
+    import oracle
+    lib = oracle.load()
+    t = time.perf_counter()
+    oracle.lloyd_step(X64[:128], C64, s.dtype, lib)
+    per_row = (time.perf_counter() - t) / 128
+    n = int(max(64, min(X64.shape[0], per_step / max(per_row, 1e-9))))
+    for _ in range(args.warmup):
+        oracle.lloyd_step(X64[:n], C64, s.dtype, lib)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.lloyd_step(X64[:n], C64, s.dtype, lib)
+    dt = time.perf_counter() - t
+    value = args.steps * n / (s.N * s.B * dt)
+    out = {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": args.workload, "N": s.N, "D": s.D, "K": s.K, "B": s.B, "dtype": s.dtype,
+                      "step": "one Lloyd iteration of the fp64 CPU oracle on a row sample"},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "kind": "oracle",
+                            "cores": oracle.num_threads(),
+                            "sample": f"{n} of {s.N * s.B} rows per step against all {s.K} centroids, "
+                                      f"scaled linearly in N"},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    del torch
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default="embed_f16")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu", dest="cpu", action="store_false")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

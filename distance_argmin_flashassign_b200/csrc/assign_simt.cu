@@ -1,0 +1,95 @@
+// assign_simt.cu -- CUDA-core assignment stage (fused distance + argmin).
+//
+// Serves fp32 inputs and every shape the tensor-core kernel does not take.
+// Like the tensor-core kernel it never writes the N x K distances to memory
+// (FlashAssign, Flash-KMeans abstract): each thread owns one point, streams
+// the centroids through shared memory in tiles of 32, keeps the 32 partial
+// squared distances in registers and folds them into a running (min, argmin)
+// in ascending centroid order, so ties go to the lowest index.  The distance
+// is the direct difference sum_j (x_j - c_j)^2 in fp32.
+#include "fk_internal.h"
+
+namespace fk {
+
+constexpr int kSimtRows = 128;  // points per block (one per thread)
+constexpr int kSimtTileK = 32;  // centroids per shared-memory tile
+
+template <typename T, int DCH>
+__global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restrict__ X,
+                                                                const T *__restrict__ C, int N,
+                                                                int D, int K,
+                                                                int32_t *__restrict__ labels,
+                                                                float *__restrict__ mindist) {
+  __shared__ float cs[kSimtTileK][DCH + 1];
+  const int b = blockIdx.y;
+  const int row = blockIdx.x * kSimtRows + threadIdx.x;
+  const bool valid = row < N;
+  const T *xrow = X + ((size_t)b * N + (valid ? row : 0)) * D;
+  const T *Cb = C + (size_t)b * K * D;
+
+  float best = __int_as_float(0x7f800000);
+  int bidx = 0;
+  for (int k0 = 0; k0 < K; k0 += kSimtTileK) {
+    float acc[kSimtTileK];
+#pragma unroll
+    for (int t = 0; t < kSimtTileK; ++t) acc[t] = 0.f;
+    for (int d0 = 0; d0 < D; d0 += DCH) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < kSimtTileK * DCH; e += kSimtRows) {
+        const int kk = e / DCH, dd = e % DCH;
+        const int k = k0 + kk, d = d0 + dd;
+        cs[kk][dd] = (k < K && d < D) ? to_f32<T>(Cb[(size_t)k * D + d]) : 0.f;
+      }
+      __syncthreads();
+      float xv[DCH];
+#pragma unroll
+      for (int dd = 0; dd < DCH; ++dd) xv[dd] = (valid && d0 + dd < D) ? to_f32<T>(xrow[d0 + dd]) : 0.f;
+#pragma unroll 4
+      for (int t = 0; t < kSimtTileK; ++t) {
+        float a = acc[t];
+#pragma unroll
+        for (int dd = 0; dd < DCH; ++dd) {
+          const float u = xv[dd] - cs[t][dd];
+          a = fmaf(u, u, a);
+        }
+        acc[t] = a;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kSimtTileK; ++t) {
+      if (k0 + t < K && acc[t] < best) {
+        best = acc[t];
+        bidx = k0 + t;
+      }
+    }
+  }
+  if (valid) {
+    labels[(size_t)b * N + row] = bidx;
+    if (mindist) mindist[(size_t)b * N + row] = best;
+  }
+}
+
+template <typename T>
+static cudaError_t launch_t(const void *X, const void *C, int B, int N, int D, int K, int32_t *labels,
+                            float *mindist, cudaStream_t s) {
+  dim3 grid((N + kSimtRows - 1) / kSimtRows, B);
+  if (D <= 32)
+    assign_simt_kernel<T, 32><<<grid, kSimtRows, 0, s>>>((const T *)X, (const T *)C, N, D, K, labels,
+                                                         mindist);
+  else
+    assign_simt_kernel<T, 64><<<grid, kSimtRows, 0, s>>>((const T *)X, (const T *)C, N, D, K, labels,
+                                                         mindist);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
+                               int32_t *labels, float *mindist, cudaStream_t s) {
+  switch (dt) {
+    case kF32: return launch_t<float>(X, C, B, N, D, K, labels, mindist, s);
+    case kF16: return launch_t<__half>(X, C, B, N, D, K, labels, mindist, s);
+    default: return launch_t<__nv_bfloat16>(X, C, B, N, D, K, labels, mindist, s);
+  }
+}
+
+}  // namespace fk

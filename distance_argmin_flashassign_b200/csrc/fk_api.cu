@@ -1,0 +1,526 @@
+// fk_api.cu -- the C ABI of libfk (see include/fk.h): argument checks, the
+// per-device state (SM count, status word, scratch cache), dispatch of the
+// assignment kernel, the Lloyd drivers and the out-of-core driver.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+
+#include "../../include/fk.h"
+#include "fk_internal.h"
+
+namespace fk {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+static std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+static std::atomic<int> g_assign_path{0};
+
+static thread_local fk_status t_last = FK_OK;
+static thread_local std::string t_msg;
+
+static fk_status fail(fk_status s, const std::string &msg) {
+  t_last = s;
+  t_msg = msg;
+  return s;
+}
+
+static fk_status cuda_fail(cudaError_t e, const char *where) {
+  const fk_status s = e == cudaErrorMemoryAllocation ? FK_ERR_OOM : FK_ERR_CUDA;
+  return fail(s, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+struct Scratch {
+  void *ptr = nullptr;
+  size_t bytes = 0;
+};
+
+struct DevState {
+  std::mutex mu;
+  bool ready = false;
+  int sms = 0;
+  int *status = nullptr;
+  std::map<cudaStream_t, Scratch> scratch;
+};
+constexpr int kMaxDevices = 64;
+static DevState g_dev[kMaxDevices];
+
+static fk_status device_state(DevState **out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FK_ERR_UNSUPPORTED, "device index out of range");
+  DevState &d = g_dev[dev];
+  std::lock_guard<std::mutex> g(d.mu);
+  if (!d.ready) {
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaMalloc(&d.status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status)");
+    e = cudaMemset(d.status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+    d.ready = true;
+  }
+  *out = &d;
+  return FK_OK;
+}
+
+static DevCtl ctl_of(const DevState &d) { return DevCtl{d.status, g_timeout_ns.load()}; }
+
+// Scratch for (device, stream), grown with stream-ordered allocation.
+static fk_status scratch(DevState &d, cudaStream_t s, size_t need, void **out) {
+  std::lock_guard<std::mutex> g(d.mu);
+  Scratch &w = d.scratch[s];
+  if (w.bytes < need) {
+    if (w.ptr) cudaFreeAsync(w.ptr, s);
+    w.ptr = nullptr;
+    w.bytes = 0;
+    const size_t want = need + need / 4 + 4096;
+    cudaError_t e = cudaMallocAsync(&w.ptr, want, s);
+    if (e != cudaSuccess) {
+      w.ptr = nullptr;
+      cudaGetLastError();
+      return cuda_fail(e, "cudaMallocAsync(scratch)");
+    }
+    w.bytes = want;
+  }
+  *out = w.ptr;
+  return FK_OK;
+}
+
+static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+
+static bool valid_dtype(fk_dtype dt) { return dt == FK_F32 || dt == FK_F16 || dt == FK_BF16; }
+
+static fk_status check_sizes(int B, int64_t N, int D, int K, fk_dtype dt) {
+  if (!valid_dtype(dt)) return fail(FK_ERR_INVALID_ARG, "unknown dtype");
+  if (B < 1 || B > 65535) return fail(FK_ERR_INVALID_ARG, "B must be in [1, 65535]");
+  if (N < 0) return fail(FK_ERR_INVALID_ARG, "N must be >= 0");
+  if (D < 1 || D > 1024) return fail(FK_ERR_INVALID_ARG, "D must be in [1, 1024]");
+  if (K < 1) return fail(FK_ERR_INVALID_ARG, "K must be >= 1");
+  if ((long long)B * N >= (1ll << 31)) return fail(FK_ERR_INVALID_ARG, "B*N must be < 2^31");
+  if ((long long)B * K > (1ll << 22)) return fail(FK_ERR_INVALID_ARG, "B*K must be <= 2^22");
+  return FK_OK;
+}
+
+// 1 = tensor-core kernel, 2 = CUDA-core kernel.
+static int choose_path(DType dt, int D) {
+  const int forced = g_assign_path.load();
+  if (forced == 2) return 2;
+  if (forced == 1) return tc_shape_ok(dt, D) ? 1 : -1;
+  return tc_shape_ok(dt, D) ? 1 : 2;
+}
+
+// Assignment of B problems.  cn (B*Kpad norms of C) may be null, in which
+// case the tensor path computes it into scratch at `cn_ws`.
+static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
+                            const float *cn, float *cn_ws, int32_t *labels, float *mindist,
+                            cudaStream_t s) {
+  const int path = choose_path(dt, D);
+  if (path < 0) return fail(FK_ERR_UNSUPPORTED, "tensor-core path forced for an unsupported shape");
+  if (path == 1 && tc_aligned(X, C)) {
+    const int Kpad = pad_k(K);
+    if (!cn) {
+      cudaError_t e = launch_norms(dt, C, B, K, Kpad, D, cn_ws, s);
+      if (e != cudaSuccess) return cuda_fail(e, "norms kernel");
+      cn = cn_ws;
+    }
+    cudaError_t e = launch_assign_tc(dt, X, C, cn, B, N, D, K, Kpad, labels, mindist, ctl_of(d), d.sms, s);
+    if (e == cudaSuccess) return FK_OK;
+    if (e != cudaErrorNotSupported) return cuda_fail(e, "tensor-core assign kernel");
+    cudaGetLastError();
+    if (g_assign_path.load() == 1) return fail(FK_ERR_UNSUPPORTED, "tensor maps could not be encoded");
+  } else if (path == 1 && g_assign_path.load() == 1) {
+    return fail(FK_ERR_UNSUPPORTED, "tensor-core path needs 16-byte aligned X and C");
+  }
+  cudaError_t e = launch_assign_simt(dt, X, C, B, N, D, K, labels, mindist, s);
+  if (e != cudaSuccess) return cuda_fail(e, "CUDA-core assign kernel");
+  return FK_OK;
+}
+
+static fk_status read_status(DevState &d, cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int h = 0;
+  e = cudaMemcpy(&h, d.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (h != 0) {
+    cudaMemset(d.status, 0, sizeof(int));
+    return fail((fk_status)h, h == FK_ERR_TIMEOUT ? "a device-side wait exceeded its time limit"
+                              : h == FK_ERR_BAD_LABEL ? "a label outside [0, K) was given to the update"
+                                                      : "device-side error");
+  }
+  return FK_OK;
+}
+
+// ------------------------------------------------------------ wait probe --
+__global__ void wait_probe_kernel(DevCtl ctl) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, ctl);  // nothing ever arrives
+}
+
+cudaError_t launch_wait_probe(DevCtl ctl, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(ctl);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fk
+
+using namespace fk;
+
+// =================================================================== ABI ===
+extern "C" {
+
+fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C, int K,
+                            int32_t *labels, float *mindist, fk_stream_t stream) {
+  fk_status st = check_sizes(B, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (N == 0) return FK_OK;
+  if (!X || !C || !labels) return fail(FK_ERR_INVALID_ARG, "X, C and labels must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, al256((size_t)B * pad_k(K) * 4), &ws)) != FK_OK) return st;
+  return run_assign(*d, (DType)dt, X, B, (int)N, D, C, K, nullptr, (float *)ws, labels, mindist, s);
+}
+
+fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, int32_t *labels,
+                    float *mindist, fk_stream_t stream) {
+  return fk_assign_batched(X, 1, N, D, dt, C, K, labels, mindist, stream);
+}
+
+int64_t fk_norms_len(int B, int K) {
+  if (B < 1 || K < 1) return 0;
+  return (int64_t)B * pad_k(K);
+}
+
+fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt, float *norms,
+                               fk_stream_t stream) {
+  fk_status st = check_sizes(B, 0, D, K, dt);
+  if (st != FK_OK) return st;
+  if (!C32 || !C_dt || !norms) return fail(FK_ERR_INVALID_ARG, "C32, C_dt and norms must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const DType t = (DType)dt;
+  cudaError_t e;
+  if (t == kF32 && C_dt == (const void *)C32)
+    e = launch_norms(t, C32, B, K, pad_k(K), D, norms, s);
+  else
+    e = launch_round_norms(t, C32, B, K, pad_k(K), D, C_dt, norms, s);
+  if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
+  return FK_OK;
+}
+
+fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt, int K,
+                             const float *norms, int32_t *labels, float *mindist, fk_stream_t stream) {
+  fk_status st = check_sizes(B, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (N == 0) return FK_OK;
+  if (!X || !C_dt || !labels || !norms) return fail(FK_ERR_INVALID_ARG, "X, C_dt, norms and labels must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  return run_assign(*d, (DType)dt, X, B, (int)N, D, C_dt, K, norms, nullptr, labels, mindist, (cudaStream_t)stream);
+}
+
+fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t N, int D, fk_dtype dt,
+                            int K, float *C, int32_t *counts, fk_stream_t stream) {
+  fk_status st = check_sizes(B, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (!C) return fail(FK_ERR_INVALID_ARG, "C must not be NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) {
+    if (counts) {
+      cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)B * K * 4, s);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(counts)");
+    }
+    return FK_OK;
+  }
+  if (!X || !labels) return fail(FK_ERR_INVALID_ARG, "X and labels must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  const size_t need = update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D);
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, need, &ws)) != FK_OK) return st;
+  UpdateArgs a{};
+  a.dt = (DType)dt;
+  a.X = X;
+  a.labels = labels;
+  a.B = B;
+  a.N = (int)N;
+  a.D = D;
+  a.K = K;
+  a.C = C;
+  a.counts = counts;
+  a.mode = kMean;
+  cudaError_t e = launch_update(a, ws, need, ctl_of(*d), d->sms, s);
+  if (e != cudaSuccess) return cuda_fail(e, "update kernels");
+  return FK_OK;
+}
+
+fk_status fk_update(const void *X, const int32_t *labels, int64_t N, int D, fk_dtype dt, int K, float *C,
+                    int32_t *counts, fk_stream_t stream) {
+  return fk_update_batched(X, labels, 1, N, D, dt, K, C, counts, stream);
+}
+
+fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, float *C, int K,
+                           int32_t *labels, float *mindist, int32_t *counts, int iters, fk_stream_t stream) {
+  fk_status st = check_sizes(B, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (iters < 1) return fail(FK_ERR_INVALID_ARG, "iters must be >= 1");
+  if (!C) return fail(FK_ERR_INVALID_ARG, "C must not be NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (N == 0) return fk_update_batched(X, labels, B, 0, D, dt, K, C, counts, stream);
+  if (!X || !labels) return fail(FK_ERR_INVALID_ARG, "X and labels must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  const DType t = (DType)dt;
+  const int Kpad = pad_k(K);
+  const size_t upd = al256(update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D));
+  const size_t cnb = al256((size_t)B * Kpad * 4);
+  const size_t cdb = t == kF32 ? 0 : al256((size_t)B * K * D * dtype_size(t));
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, upd + cnb + cdb, &ws)) != FK_OK) return st;
+  float *cn = (float *)((char *)ws + upd);
+  void *Cdt = t == kF32 ? (void *)C : (void *)((char *)ws + upd + cnb);
+
+  UpdateArgs a{};
+  a.dt = t;
+  a.X = X;
+  a.labels = labels;
+  a.B = B;
+  a.N = (int)N;
+  a.D = D;
+  a.K = K;
+  a.C = C;
+  a.counts = counts;
+  a.mode = kMean;
+  for (int it = 0; it < iters; ++it) {
+    if (t != kF32) {  // fp32 runs on the CUDA-core kernel, which needs no norms
+      cudaError_t e = launch_round_norms(t, C, B, K, Kpad, D, Cdt, cn, s);
+      if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
+    }
+    st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, labels, it == iters - 1 ? mindist : nullptr, s);
+    if (st != FK_OK) return st;
+    cudaError_t e = launch_update(a, ws, upd, ctl_of(*d), d->sms, s);
+    if (e != cudaSuccess) return cuda_fail(e, "update kernels");
+  }
+  return read_status(*d, s);
+}
+
+fk_status fk_lloyd(const void *X, int64_t N, int D, fk_dtype dt, float *C, int K, int32_t *labels,
+                   float *mindist, int32_t *counts, int iters, fk_stream_t stream) {
+  return fk_lloyd_batched(X, 1, N, D, dt, C, K, labels, mindist, counts, iters, stream);
+}
+
+fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float *C_host, int K,
+                       int32_t *labels_host, int32_t *counts_host, int iters, int64_t chunk_rows,
+                       fk_stream_t stream) {
+  fk_status st = check_sizes(1, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (iters < 1) return fail(FK_ERR_INVALID_ARG, "iters must be >= 1");
+  if (chunk_rows < 1) return fail(FK_ERR_INVALID_ARG, "chunk_rows must be >= 1");
+  if (!C_host) return fail(FK_ERR_INVALID_ARG, "C_host must not be NULL");
+  if (N == 0) {
+    if (counts_host) memset(counts_host, 0, (size_t)K * 4);
+    return FK_OK;
+  }
+  if (!X_host) return fail(FK_ERR_INVALID_ARG, "X_host must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  const DType t = (DType)dt;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t rows = chunk_rows < N ? chunk_rows : N;
+  const int64_t nchunks = (N + rows - 1) / rows;
+  const size_t es = dtype_size(t);
+  const int Kpad = pad_k(K);
+
+  // device buffers owned by this call
+  const size_t b_ring = al256((size_t)rows * D * es), b_lab = al256((size_t)rows * 4);
+  const size_t b_c32 = al256((size_t)K * D * 4), b_cdt = t == kF32 ? 0 : al256((size_t)K * D * es);
+  const size_t b_cn = al256((size_t)Kpad * 4), b_acc = al256((size_t)K * D * 8);
+  const size_t b_cnt = al256((size_t)K * 8), b_counts = al256((size_t)K * 4);
+  const size_t b_upd = al256(update_workspace_bytes(rows, K, D));
+  const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd;
+
+  cudaStream_t cs = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  char *mem = nullptr;
+  fk_status rc = FK_OK;
+  cudaError_t e;
+#define FK_TRY(call, what, code)        \
+  do {                                  \
+    e = (call);                         \
+    if (e != cudaSuccess) {             \
+      rc = code == FK_ERR_CUDA ? cuda_fail(e, what) : fail(code, std::string(what) + ": " + cudaGetErrorString(e)); \
+      goto done;                        \
+    }                                   \
+  } while (0)
+  {
+    FK_TRY(cudaMallocAsync((void **)&mem, total, s), "cudaMallocAsync(out-of-core buffers)", FK_ERR_OOM);
+    FK_TRY(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking), "cudaStreamCreate", FK_ERR_CUDA);
+    for (int i = 0; i < 2; ++i) {
+      FK_TRY(cudaEventCreateWithFlags(&ready[i], cudaEventDisableTiming), "cudaEventCreate", FK_ERR_CUDA);
+      FK_TRY(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming), "cudaEventCreate", FK_ERR_CUDA);
+    }
+    char *p = mem;
+    char *ring[2] = {p, p + b_ring};
+    p += 2 * b_ring;
+    int32_t *lab[2] = {(int32_t *)p, (int32_t *)(p + b_lab)};
+    p += 2 * b_lab;
+    float *c32 = (float *)p; p += b_c32;
+    void *cdt = t == kF32 ? (void *)c32 : (void *)p; p += b_cdt;
+    float *cn = (float *)p; p += b_cn;
+    double *acc = (double *)p; p += b_acc;
+    long long *cnt = (long long *)p; p += b_cnt;
+    int32_t *cnts = (int32_t *)p; p += b_counts;
+    void *upd = (void *)p;
+
+    // Make the allocation visible to the copy stream before it is used there.
+    FK_TRY(cudaEventRecord(freed[0], s), "cudaEventRecord", FK_ERR_CUDA);
+    FK_TRY(cudaEventRecord(freed[1], s), "cudaEventRecord", FK_ERR_CUDA);
+    FK_TRY(cudaMemcpyAsync(c32, C_host, (size_t)K * D * 4, cudaMemcpyHostToDevice, s), "copy of C to the device",
+           FK_ERR_HOST_IO);
+    UpdateArgs a{};
+    a.dt = t;
+    a.B = 1;
+    a.D = D;
+    a.K = K;
+    a.acc = acc;
+    a.cnt = cnt;
+    a.mode = kAccumulate;
+    for (int it = 0; it < iters; ++it) {
+      FK_TRY(cudaMemsetAsync(acc, 0, (size_t)K * D * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
+      FK_TRY(cudaMemsetAsync(cnt, 0, (size_t)K * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
+      if (t != kF32)
+        FK_TRY(launch_round_norms(t, c32, 1, K, Kpad, D, cdt, cn, s), "centroid prep kernel", FK_ERR_CUDA);
+      for (int64_t c = 0; c < nchunks; ++c) {
+        const int slot = (int)(c & 1);
+        const int64_t r0 = c * rows;
+        const int nr = (int)((N - r0) < rows ? (N - r0) : rows);
+        // copy stream: chunk c into its slot once the compute that last read the slot is done
+        FK_TRY(cudaStreamWaitEvent(cs, freed[slot], 0), "cudaStreamWaitEvent", FK_ERR_CUDA);
+        FK_TRY(cudaMemcpyAsync(ring[slot], (const char *)X_host + (size_t)r0 * D * es, (size_t)nr * D * es,
+                               cudaMemcpyHostToDevice, cs),
+               "host-to-device copy of a chunk", FK_ERR_HOST_IO);
+        FK_TRY(cudaEventRecord(ready[slot], cs), "cudaEventRecord", FK_ERR_CUDA);
+        // compute stream: assign the chunk and accumulate its per-cluster sums
+        FK_TRY(cudaStreamWaitEvent(s, ready[slot], 0), "cudaStreamWaitEvent", FK_ERR_CUDA);
+        rc = run_assign(*d, t, ring[slot], 1, nr, D, cdt, K, cn, nullptr, lab[slot], nullptr, s);
+        if (rc != FK_OK) goto done;
+        if (it == iters - 1 && labels_host)
+          FK_TRY(cudaMemcpyAsync(labels_host + r0, lab[slot], (size_t)nr * 4, cudaMemcpyDeviceToHost, s),
+                 "device-to-host copy of labels", FK_ERR_HOST_IO);
+        a.X = ring[slot];
+        a.labels = lab[slot];
+        a.N = nr;
+        FK_TRY(launch_update(a, upd, b_upd, ctl_of(*d), d->sms, s), "update kernels", FK_ERR_CUDA);
+        FK_TRY(cudaEventRecord(freed[slot], s), "cudaEventRecord", FK_ERR_CUDA);
+      }
+      FK_TRY(launch_divide_accumulated(acc, cnt, K, D, c32, cnts, s), "divide kernel", FK_ERR_CUDA);
+    }
+    FK_TRY(cudaMemcpyAsync(C_host, c32, (size_t)K * D * 4, cudaMemcpyDeviceToHost, s), "copy of C to the host",
+           FK_ERR_HOST_IO);
+    if (counts_host)
+      FK_TRY(cudaMemcpyAsync(counts_host, cnts, (size_t)K * 4, cudaMemcpyDeviceToHost, s),
+             "copy of counts to the host", FK_ERR_HOST_IO);
+    rc = read_status(*d, s);
+  }
+done:
+#undef FK_TRY
+  if (cs) {
+    cudaStreamSynchronize(cs);
+    cudaStreamDestroy(cs);
+  }
+  if (mem) {
+    cudaFreeAsync(mem, s);
+    cudaStreamSynchronize(s);
+  }
+  for (int i = 0; i < 2; ++i) {
+    if (ready[i]) cudaEventDestroy(ready[i]);
+    if (freed[i]) cudaEventDestroy(freed[i]);
+  }
+  return rc;
+}
+
+fk_status fk_sync(fk_stream_t stream) {
+  DevState *d;
+  fk_status st = device_state(&d);
+  if (st != FK_OK) return st;
+  return read_status(*d, (cudaStream_t)stream);
+}
+
+const char *fk_status_string(fk_status s) {
+  switch (s) {
+    case FK_OK: return "ok";
+    case FK_ERR_INVALID_ARG: return "invalid argument";
+    case FK_ERR_UNSUPPORTED: return "unsupported request";
+    case FK_ERR_CUDA: return "CUDA error";
+    case FK_ERR_OOM: return "out of memory";
+    case FK_ERR_TIMEOUT: return "device-side wait timed out";
+    case FK_ERR_HOST_IO: return "host/device copy failed";
+    case FK_ERR_BAD_LABEL: return "label outside [0, K)";
+    default: return "unknown status";
+  }
+}
+
+fk_status fk_get_last_error(void) { return t_last; }
+const char *fk_last_error_message(void) { return t_msg.c_str(); }
+uint64_t fk_launch_count(void) { return g_launches.load(); }
+
+int fk_assign_path(int64_t N, int D, fk_dtype dt, int K, int B) {
+  if (!valid_dtype(dt) || B < 1 || N < 0 || D < 1 || D > 1024 || K < 1) return FK_ERR_INVALID_ARG;
+  return choose_path((DType)dt, D);
+}
+
+fk_status fk_set_assign_path(int path) {
+  if (path < 0 || path > 2) return fail(FK_ERR_INVALID_ARG, "path must be 0, 1 or 2");
+  g_assign_path.store(path);
+  return FK_OK;
+}
+
+fk_status fk_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns == 0 ? 2000000000ull : (unsigned long long)ns);
+  return FK_OK;
+}
+
+fk_status fk_debug_wait_timeout(uint64_t ns, fk_stream_t stream) {
+  DevState *d;
+  fk_status st = device_state(&d);
+  if (st != FK_OK) return st;
+  DevCtl c = ctl_of(*d);
+  c.timeout_ns = ns;
+  cudaError_t e = launch_wait_probe(c, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe kernel");
+  return read_status(*d, (cudaStream_t)stream);
+}
+
+fk_status fk_release_workspace(void) {
+  DevState *d;
+  fk_status st = device_state(&d);
+  if (st != FK_OK) return st;
+  std::lock_guard<std::mutex> g(d->mu);
+  for (auto &kv : d->scratch) {
+    if (kv.second.ptr) cudaFreeAsync(kv.second.ptr, kv.first);
+  }
+  d->scratch.clear();
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  return FK_OK;
+}
+
+int fk_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// fk_internal.h -- host-side interface between the C ABI (fk_api.cu) and the
+// kernel files.  Every launcher enqueues on `s`, counts its launches and
+// returns the CUDA error of the launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "fk_common.cuh"
+
+namespace fk {
+
+void count_launches(int n);
+
+constexpr int kCentroidPad = 256;  // centroid tile of the tensor-core kernel
+inline int pad_k(int K) { return (K + kCentroidPad - 1) / kCentroidPad * kCentroidPad; }
+inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
+
+// ---- prep.cu: centroid norms (row norms of the assignment stage) ----------
+// cn[b*Kpad + j] = |C[b][j]|^2 in fp32 for j < K, +inf for K <= j < Kpad.
+cudaError_t launch_norms(DType dt, const void *C, int B, int K, int Kpad, int D, float *cn,
+                         cudaStream_t s);
+// Cdt = C32 rounded to dt (round-to-nearest-even) and cn = norms of Cdt.
+cudaError_t launch_round_norms(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
+                               float *cn, cudaStream_t s);
+
+// ---- assign_simt.cu: CUDA-core assignment (any dtype, any D) --------------
+cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
+                               int32_t *labels, float *mindist, cudaStream_t s);
+
+// ---- assign_tc.cu: tcgen05 assignment (fp16/bf16, D % 8 == 0, D <= 128) --
+bool tc_shape_ok(DType dt, int D);
+bool tc_aligned(const void *X, const void *C);
+// Returns cudaErrorNotSupported if the tensor maps could not be encoded.
+cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *cn, int B, int N,
+                             int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
+                             int num_sms, cudaStream_t s);
+
+// ---- update.cu: sort-inverse update ---------------------------------------
+enum UpdateMode : int { kMean = 0, kAccumulate = 1 };
+struct UpdateArgs {
+  DType dt;
+  const void *X;          // B*N rows of D elements
+  const int32_t *labels;  // B*N
+  int B, N, D, K;
+  float *C;               // kMean: B*K x D fp32 in/out
+  int32_t *counts;        // kMean: B*K or null
+  double *acc;            // kAccumulate: B*K x D fp64 running sums
+  long long *cnt;         // kAccumulate: B*K running counts
+  UpdateMode mode;
+};
+size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D);
+cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl ctl,
+                          int num_sms, cudaStream_t s);
+// C[k] = acc[k] / cnt[k] (fp32) where cnt[k] > 0, counts[k] = cnt[k]; acc and
+// cnt are reset to zero.
+cudaError_t launch_divide_accumulated(double *acc, long long *cnt, int Ktot, int D, float *C,
+                                      int32_t *counts, cudaStream_t s);
+
+// ---- fk_api.cu: timeout self-test kernel -----------------------------------
+cudaError_t launch_wait_probe(DevCtl ctl, cudaStream_t s);
+
+}  // namespace fk

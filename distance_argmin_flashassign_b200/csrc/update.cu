@@ -1,0 +1,571 @@
+// update.cu -- sort-inverse centroid update.
+//
+// Flash-KMeans (arXiv 2603.09229, abstract) replaces the per-point atomic
+// scatter of the update stage by an explicitly built inverse mapping and
+// segment-level localized reductions.  Here:
+//
+//   1. stable LSD radix sort of the cluster ids (11-bit digits, one pass for
+//      up to 2,048 clusters, two for up to 2^22): per-tile digit histograms,
+//      a per-digit scan over tiles, and a scatter whose within-tile ranks come
+//      from warp-level match_any -- the sorted point ids are the inverse map
+//      (cluster -> its points);
+//   2. segment offsets by a lower-bound search of every cluster id in the
+//      sorted ids;
+//   3. segmented sums: the sorted order is cut into equal chunks of R
+//      positions, one warp per chunk, so a hot cluster (Zipf skew) is spread
+//      over many warps instead of serialising on one address.  A warp gathers
+//      its rows coalesced (each row is read as one contiguous vector per
+//      lane), accumulates in fp32 registers and writes a segment that lies
+//      wholly inside its chunk straight to the output; the two boundary
+//      segments of a chunk go to partial slots;
+//   4. finalize: per cluster, partials of chunk-crossing segments are summed
+//      in a fixed order and divided by the count; empty clusters are left
+//      untouched.  No global atomics anywhere, so results are deterministic.
+//
+// Batched problems are one problem over B*K clusters: point (b, i) gets key
+// b*K + label.
+#include "fk_internal.h"
+
+namespace fk {
+
+constexpr int kSortThreads = 256;
+constexpr int kSortItems = 16;
+constexpr int kSortTile = kSortThreads * kSortItems;  // 4096 keys per tile
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kMaxDigitBits = 11;
+constexpr int kMaxBins = 1 << kMaxDigitBits;
+
+struct SortPlan {
+  int npass;
+  int shift[2], bits[2];
+  int T;  // tiles
+};
+
+static int ceil_log2(long long v) {
+  int b = 0;
+  while ((1ll << b) < v) ++b;
+  return b;
+}
+
+static SortPlan plan_sort(long long Ntot, long long Ktot) {
+  SortPlan p{};
+  int bits = ceil_log2(Ktot);
+  if (bits < 1) bits = 1;
+  p.npass = (bits + kMaxDigitBits - 1) / kMaxDigitBits;
+  const int w = (bits + p.npass - 1) / p.npass;
+  int sh = 0;
+  for (int i = 0; i < p.npass; ++i) {
+    p.shift[i] = sh;
+    p.bits[i] = (bits - sh) < w ? (bits - sh) : w;
+    sh += p.bits[i];
+  }
+  p.T = (int)((Ntot + kSortTile - 1) / kSortTile);
+  return p;
+}
+
+static int chunk_rows_R(long long Ntot) {
+  long long R = (Ntot / 8192 + 31) / 32 * 32;
+  return (int)(R < 256 ? 256 : R);
+}
+
+// --------------------------------------------------------------- sorting --
+__device__ __forceinline__ int first_key(const int32_t *__restrict__ labels, int pos, int N, int K,
+                                         int B, int *status) {
+  int lab = labels[pos];
+  if ((unsigned)lab >= (unsigned)K) {
+    record_status(status, kStBadLabel);
+    lab = 0;
+  }
+  return B > 1 ? (pos / N) * K + lab : lab;
+}
+
+template <bool FIRST>
+__global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t *__restrict__ keys, int Ntot,
+                                                                  int N, int K, int B, int shift, int nbins,
+                                                                  int T, int *__restrict__ H,
+                                                                  int *status) {
+  __shared__ int hist[kMaxBins + 1];
+  for (int i = threadIdx.x; i <= nbins; i += kSortThreads) hist[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int base = blockIdx.x * kSortTile;
+#pragma unroll 4
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * kSortThreads + threadIdx.x;
+    int d = nbins;  // spare bin for positions past the end
+    if (pos < Ntot) {
+      const int key = FIRST ? first_key(keys, pos, N, K, B, status) : keys[pos];
+      d = (key >> shift) & (nbins - 1);
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    if (lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nbins; i += kSortThreads) H[(size_t)i * T + blockIdx.x] = hist[i];
+}
+
+// In place: row d of H becomes the exclusive prefix over tiles; totals[d] = row sum.
+__global__ void __launch_bounds__(256) scan_rows_kernel(int *__restrict__ H, int T, int nbins,
+                                                        int *__restrict__ totals) {
+  const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (w >= nbins) return;
+  int *row = H + (size_t)w * T;
+  int carry = 0;
+  for (int t0 = 0; t0 < T; t0 += 32) {
+    const int v = (t0 + lane < T) ? row[t0 + lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (t0 + lane < T) row[t0 + lane] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) totals[w] = carry;
+}
+
+template <bool FIRST>
+__global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
+    const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in, int32_t *__restrict__ keys_out,
+    int32_t *__restrict__ vals_out, int Ntot, int N, int K, int B, int shift, int nbins, int T,
+    const int *__restrict__ H, const int *__restrict__ totals, int *status) {
+  extern __shared__ int sh[];
+  int *dbase = sh;                                                   // [nbins]
+  int *wsum = sh + nbins;                                            // [8]
+  uint16_t *wcnt = reinterpret_cast<uint16_t *>(sh + nbins + 8);     // [8][nbins + 1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int stride = nbins + 1;
+
+  // digit base of this tile = exclusive scan of digit totals + tile prefix
+  const int per = (nbins + kSortThreads - 1) / kSortThreads;
+  int s = 0;
+  for (int i = 0; i < per; ++i) {
+    const int d = tid * per + i;
+    if (d < nbins) s += totals[d];
+  }
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  for (int i = tid; i < kSortWarps * stride; i += kSortThreads) wcnt[i] = 0;
+  __syncthreads();
+  int run = incl - s;
+  for (int w = 0; w < warp; ++w) run += wsum[w];
+  for (int i = 0; i < per; ++i) {
+    const int d = tid * per + i;
+    if (d < nbins) {
+      dbase[d] = run + H[(size_t)d * T + blockIdx.x];
+      run += totals[d];
+    }
+  }
+
+  // stable ranks within each warp's 512 consecutive keys
+  int keyr[kSortItems], valr[kSortItems], locr[kSortItems];
+  const int base = blockIdx.x * kSortTile + warp * (kSortItems * 32);
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint16_t *mycnt = wcnt + warp * stride;
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * 32 + lane;
+    int d = nbins, key = 0, val = 0;
+    if (pos < Ntot) {
+      key = FIRST ? first_key(keys_in, pos, N, K, B, status) : keys_in[pos];
+      val = FIRST ? pos : vals_in[pos];
+      d = (key >> shift) & (nbins - 1);
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    const int c = mycnt[d];
+    __syncwarp();
+    if (lane == __ffs(peers) - 1) mycnt[d] = (uint16_t)(c + __popc(peers));
+    __syncwarp();
+    keyr[it] = key;
+    valr[it] = val;
+    locr[it] = c + __popc(peers & lt_mask);
+  }
+  __syncthreads();
+  for (int d = tid; d < nbins; d += kSortThreads) {
+    int r = 0;
+    for (int w = 0; w < kSortWarps; ++w) {
+      const int t = wcnt[w * stride + d];
+      wcnt[w * stride + d] = (uint16_t)r;
+      r += t;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * 32 + lane;
+    if (pos < Ntot) {
+      const int d = (keyr[it] >> shift) & (nbins - 1);
+      const int o = dbase[d] + mycnt[d] + locr[it];
+      keys_out[o] = keyr[it];
+      vals_out[o] = valr[it];
+    }
+  }
+}
+
+// off[k] = first position of key >= k in the sorted keys, k in [0, Ktot].
+__global__ void __launch_bounds__(256) seg_offsets_kernel(const int32_t *__restrict__ skeys, int Ntot,
+                                                          int Ktot, int *__restrict__ off) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k > Ktot) return;
+  int lo = 0, hi = Ntot;
+  while (lo < hi) {
+    const int mid = lo + ((hi - lo) >> 1);
+    if (skeys[mid] < k) lo = mid + 1; else hi = mid;
+  }
+  off[k] = lo;
+}
+
+// ------------------------------------------------------- segmented sums --
+template <typename T> struct Vec;
+template <> struct Vec<float> {
+  template <int N> __device__ static void load(const float *p, float *v) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 4; ++i) {
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(p) + i);
+        v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+      }
+    } else if constexpr (N == 2) {
+      const float2 w = __ldg(reinterpret_cast<const float2 *>(p));
+      v[0] = w.x; v[1] = w.y;
+    } else {
+      v[0] = __ldg(p);
+    }
+  }
+};
+__device__ __forceinline__ void unpack_half2(uint32_t w, float *v) {
+  const __half2 h = *reinterpret_cast<const __half2 *>(&w);
+  v[0] = __low2float(h);
+  v[1] = __high2float(h);
+}
+__device__ __forceinline__ void unpack_bf162(uint32_t w, float *v) {
+  v[0] = __uint_as_float(w << 16);
+  v[1] = __uint_as_float(w & 0xffff0000u);
+}
+template <typename T, bool BF> struct Vec16 {
+  template <int N> __device__ static void load(const T *p, float *v) {
+    auto up = [](uint32_t w, float *o) { if (BF) unpack_bf162(w, o); else unpack_half2(w, o); };
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+        up(w.x, v + 8 * i); up(w.y, v + 8 * i + 2); up(w.z, v + 8 * i + 4); up(w.w, v + 8 * i + 6);
+      }
+    } else if constexpr (N == 4) {
+      const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+      up(w.x, v); up(w.y, v + 2);
+    } else if constexpr (N == 2) {
+      up(__ldg(reinterpret_cast<const unsigned int *>(p)), v);
+    } else {
+      v[0] = to_f32<T>(p[0]);
+    }
+  }
+};
+template <> struct Vec<__half> : Vec16<__half, false> {};
+template <> struct Vec<__nv_bfloat16> : Vec16<__nv_bfloat16, true> {};
+
+// CONTIG: lane l owns dims [l*NACC, l*NACC + NACC) (D == 32*NACC, vector loads);
+// otherwise lane l owns dims l + 32*a, a < NACC, masked by D.
+template <typename T, int NACC, bool CONTIG, int MODE>
+__global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, int D,
+                                                     const int32_t *__restrict__ perm,
+                                                     const int32_t *__restrict__ skeys, int Ntot, int R,
+                                                     float *__restrict__ C, double *__restrict__ acc,
+                                                     float *__restrict__ parts) {
+  constexpr int PF = NACC <= 4 ? 8 : (NACC <= 8 ? 4 : (NACC <= 16 ? 2 : 1));  // rows in flight
+  const int lane = threadIdx.x & 31;
+  const long long wq = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long p0l = wq * R;
+  if (p0l >= Ntot) return;
+  const int p0 = (int)p0l;
+  const int p1 = (Ntot - p0) < R ? Ntot : p0 + R;
+  const int kfirst = skeys[p0];
+  const bool split_start = p0 > 0 && skeys[p0 - 1] == kfirst;
+  const bool split_end = p1 < Ntot && skeys[p1] == skeys[p1 - 1];
+
+  float a[NACC];
+#pragma unroll
+  for (int i = 0; i < NACC; ++i) a[i] = 0.f;
+  int cur = kfirst, s = p0;
+
+  auto dim_of = [&](int i) { return CONTIG ? lane * NACC + i : lane + 32 * i; };
+  auto flush = [&](int k, int sb, int se) {
+    const bool split = (sb == p0 && split_start) || (se == p1 && split_end);
+    if (!split) {
+      if (MODE == kMean) {
+        const float fc = (float)(se - sb);
+        float *dst = C + (size_t)k * D;
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) {
+          const int d = dim_of(i);
+          if (CONTIG || d < D) dst[d] = a[i] / fc;
+        }
+      } else {
+        double *dst = acc + (size_t)k * D;
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) {
+          const int d = dim_of(i);
+          if (CONTIG || d < D) dst[d] += (double)a[i];
+        }
+      }
+    } else {
+      float *dst = parts + ((size_t)wq * 2 + (sb == p0 ? 0 : 1)) * D;
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) {
+        const int d = dim_of(i);
+        if (CONTIG || d < D) dst[d] = a[i];
+      }
+    }
+  };
+
+  for (int b0 = p0; b0 < p1; b0 += 32) {
+    const int n = (p1 - b0) < 32 ? (p1 - b0) : 32;
+    const int mk = lane < n ? skeys[b0 + lane] : 0;
+    const int mr = lane < n ? perm[b0 + lane] : 0;
+    for (int t0 = 0; t0 < n; t0 += PF) {
+      float v[PF][NACC];
+#pragma unroll
+      for (int u = 0; u < PF; ++u) {
+        const int row = __shfl_sync(0xffffffffu, mr, (t0 + u) & 31);
+        if (t0 + u < n) {
+          const T *xr = X + (size_t)row * D;
+          if (CONTIG) {
+            Vec<T>::template load<NACC>(xr + lane * NACC, v[u]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < NACC; ++i) {
+              const int d = lane + 32 * i;
+              v[u][i] = d < D ? to_f32<T>(xr[d]) : 0.f;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < PF; ++u) {
+        const int k = __shfl_sync(0xffffffffu, mk, (t0 + u) & 31);
+        if (t0 + u < n) {
+          if (k != cur) {
+            flush(cur, s, b0 + t0 + u);
+            cur = k;
+            s = b0 + t0 + u;
+#pragma unroll
+            for (int i = 0; i < NACC; ++i) a[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < NACC; ++i) a[i] += v[u][i];
+        }
+      }
+    }
+  }
+  flush(cur, s, p1);
+}
+
+// One block per cluster (grid-stride): counts, then the fixed-order sum of
+// the partials of a segment that crosses chunk borders.
+template <int MODE>
+__global__ void __launch_bounds__(512) seg_finalize_kernel(const int *__restrict__ off, int Ktot, int D, int R,
+                                                           const float *__restrict__ parts,
+                                                           float *__restrict__ C, int32_t *__restrict__ counts,
+                                                           double *__restrict__ acc, long long *__restrict__ cnt) {
+  __shared__ float red[512];
+  const int tid = threadIdx.x;
+  const int G = D >= 512 ? 1 : 512 / D;  // groups of partials summed in parallel
+  for (int k = blockIdx.x; k < Ktot; k += gridDim.x) {
+    const int s = off[k], e = off[k + 1], n = e - s;
+    if (tid == 0) {
+      if (MODE == kMean) {
+        if (counts) counts[k] = n;
+      } else {
+        cnt[k] += n;
+      }
+    }
+    if (n == 0) continue;
+    const int q0 = s / R, q1 = (e - 1) / R;
+    if (q0 == q1) continue;  // segment inside one chunk: already written
+    const int np = q1 - q0 + 1;
+    const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
+    auto part_row = [&](int i) { return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D; };
+    if (G > 1) {
+      const int g = tid / D, d = tid % D;
+      float t = 0.f;
+      if (g < G)
+        for (int i = g; i < np; i += G) t += part_row(i)[d];
+      red[tid] = t;
+      __syncthreads();
+      if (tid < D) {
+        float tot = 0.f;
+        for (int gg = 0; gg < G; ++gg) tot += red[gg * D + tid];
+        if (MODE == kMean) C[(size_t)k * D + tid] = tot / (float)n;
+        else acc[(size_t)k * D + tid] += (double)tot;
+      }
+      __syncthreads();
+    } else {
+      for (int d = tid; d < D; d += blockDim.x) {
+        float tot = 0.f;
+        for (int i = 0; i < np; ++i) tot += part_row(i)[d];
+        if (MODE == kMean) C[(size_t)k * D + d] = tot / (float)n;
+        else acc[(size_t)k * D + d] += (double)tot;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) divide_acc_kernel(const double *__restrict__ acc,
+                                                         const long long *__restrict__ cnt, int Ktot, int D,
+                                                         float *__restrict__ C, int32_t *__restrict__ counts) {
+  const size_t total = (size_t)Ktot * D;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int k = (int)(i / D);
+    const long long n = cnt[k];
+    if (n > 0) C[i] = (float)(acc[i] / (double)n);
+    if (counts && i % D == 0) counts[k] = (int32_t)n;
+  }
+}
+
+// ---------------------------------------------------------------- host ---
+static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+
+struct UpdateWs {
+  int32_t *kA, *vA, *kB, *vB;
+  int *H, *totals, *off;
+  float *parts;
+  size_t bytes;
+};
+
+static UpdateWs carve(void *base, long long Ntot, long long Ktot, int D) {
+  const SortPlan sp = plan_sort(Ntot, Ktot);
+  const int R = chunk_rows_R(Ntot);
+  const long long nchunks = (Ntot + R - 1) / R;
+  int maxbins = 0;
+  for (int i = 0; i < sp.npass; ++i) maxbins = (1 << sp.bits[i]) > maxbins ? (1 << sp.bits[i]) : maxbins;
+  UpdateWs w{};
+  char *p = (char *)base;
+  size_t o = 0;
+  auto take = [&](size_t n) { char *r = p ? p + o : nullptr; o += al256(n); return r; };
+  w.kA = (int32_t *)take((size_t)Ntot * 4);
+  w.vA = (int32_t *)take((size_t)Ntot * 4);
+  w.kB = (int32_t *)take((size_t)Ntot * 4);
+  w.vB = (int32_t *)take((size_t)Ntot * 4);
+  w.H = (int *)take((size_t)maxbins * sp.T * 4);
+  w.totals = (int *)take((size_t)maxbins * 4);
+  w.off = (int *)take((size_t)(Ktot + 1) * 4);
+  w.parts = (float *)take((size_t)nchunks * 2 * D * 4);
+  w.bytes = o;
+  return w;
+}
+
+size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D) {
+  return carve(nullptr, Ntot, Ktot, D).bytes;
+}
+
+template <typename T, int MODE>
+static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_t *skeys, int Ntot, int R,
+                          float *parts, cudaStream_t s) {
+  const long long nchunks = ((long long)Ntot + R - 1) / R;
+  const int grid = (int)((nchunks + 7) / 8);
+  const T *X = (const T *)a.X;
+  const int D = a.D;
+  const size_t es = sizeof(T);
+  const bool contig_ok = D % 32 == 0 && ((uintptr_t)a.X % 16 == 0);
+  const int nacc_c = D / 32;
+#define FK_SEG(NA, CG) \
+  segsum_kernel<T, NA, CG, MODE><<<grid, 256, 0, s>>>(X, D, perm, skeys, Ntot, R, a.C, a.acc, parts)
+  if (contig_ok && nacc_c == 1) FK_SEG(1, true);
+  else if (contig_ok && nacc_c == 2) FK_SEG(2, true);
+  else if (contig_ok && nacc_c == 4) FK_SEG(4, true);
+  else if (contig_ok && nacc_c == 8) FK_SEG(8, true);
+  else {
+    const int need = (D + 31) / 32;
+    if (need <= 1) FK_SEG(1, false);
+    else if (need <= 2) FK_SEG(2, false);
+    else if (need <= 4) FK_SEG(4, false);
+    else if (need <= 8) FK_SEG(8, false);
+    else if (need <= 16) FK_SEG(16, false);
+    else FK_SEG(32, false);
+  }
+#undef FK_SEG
+  (void)es;
+}
+
+cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl ctl, int num_sms,
+                          cudaStream_t s) {
+  const long long Ntot = (long long)a.B * a.N, Ktot = (long long)a.B * a.K;
+  if (Ntot == 0) return cudaSuccess;
+  const UpdateWs w = carve(ws, Ntot, Ktot, a.D);
+  if (w.bytes > ws_bytes) return cudaErrorInvalidValue;
+  const SortPlan sp = plan_sort(Ntot, Ktot);
+  const int N = (int)Ntot;
+  int nl = 0;
+
+  const int32_t *kin = a.labels, *vin = nullptr;
+  int32_t *kout = w.kA, *vout = w.vA;
+  for (int pass = 0; pass < sp.npass; ++pass) {
+    const int nbins = 1 << sp.bits[pass];
+    if (pass == 0)
+      radix_hist_kernel<true><<<sp.T, kSortThreads, 0, s>>>(kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
+                                                            sp.T, w.H, ctl.status);
+    else
+      radix_hist_kernel<false><<<sp.T, kSortThreads, 0, s>>>(kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
+                                                             sp.T, w.H, ctl.status);
+    scan_rows_kernel<<<(nbins + 7) / 8, 256, 0, s>>>(w.H, sp.T, nbins, w.totals);
+    const size_t shb = (size_t)(nbins + 8) * 4 + (size_t)kSortWarps * (nbins + 1) * 2;
+    if (pass == 0)
+      radix_scatter_kernel<true><<<sp.T, kSortThreads, shb, s>>>(kin, vin, kout, vout, N, a.N, a.K, a.B,
+                                                                 sp.shift[pass], nbins, sp.T, w.H,
+                                                                 w.totals, ctl.status);
+    else
+      radix_scatter_kernel<false><<<sp.T, kSortThreads, shb, s>>>(kin, vin, kout, vout, N, a.N, a.K, a.B,
+                                                                  sp.shift[pass], nbins, sp.T, w.H,
+                                                                  w.totals, ctl.status);
+    nl += 3;
+    kin = kout;
+    vin = vout;
+    kout = (kout == w.kA) ? w.kB : w.kA;
+    vout = (vout == w.vA) ? w.vB : w.vA;
+  }
+  const int32_t *skeys = kin, *perm = vin;
+  seg_offsets_kernel<<<(int)((Ktot + 1 + 255) / 256), 256, 0, s>>>(skeys, N, (int)Ktot, w.off);
+  const int R = chunk_rows_R(Ntot);
+  switch (a.dt) {
+    case kF32:
+      a.mode == kMean ? launch_segsum<float, kMean>(a, perm, skeys, N, R, w.parts, s)
+                      : launch_segsum<float, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+      break;
+    case kF16:
+      a.mode == kMean ? launch_segsum<__half, kMean>(a, perm, skeys, N, R, w.parts, s)
+                      : launch_segsum<__half, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+      break;
+    default:
+      a.mode == kMean ? launch_segsum<__nv_bfloat16, kMean>(a, perm, skeys, N, R, w.parts, s)
+                      : launch_segsum<__nv_bfloat16, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+  }
+  const int fgrid = (int)(Ktot < (long long)num_sms * 4 ? Ktot : (long long)num_sms * 4);
+  if (a.mode == kMean)
+    seg_finalize_kernel<kMean><<<fgrid, 512, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
+                                                     nullptr, nullptr);
+  else
+    seg_finalize_kernel<kAccumulate><<<fgrid, 512, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr,
+                                                           nullptr, a.acc, a.cnt);
+  nl += 3;
+  count_launches(nl);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_divide_accumulated(double *acc, long long *cnt, int Ktot, int D, float *C,
+                                      int32_t *counts, cudaStream_t s) {
+  const size_t total = (size_t)Ktot * D;
+  long long g = (long long)((total + 255) / 256);
+  if (g > 8192) g = 8192;
+  if (g < 1) g = 1;
+  divide_acc_kernel<<<(int)g, 256, 0, s>>>(acc, cnt, Ktot, D, C, counts);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fk

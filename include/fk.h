@@ -1,0 +1,252 @@
+/*
+ * fk.h -- C ABI of libfk, exact Lloyd k-means on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one "Flash-KMeans: Fast and Memory-Efficient Exact
+ * K-Means" (arXiv 2603.09229) states in its abstract: one Lloyd iteration is an
+ * assignment stage (the nearest of K centroids for each of N points in D
+ * dimensions) followed by a centroid-update stage (each centroid becomes the
+ * mean of the points assigned to it), computed exactly -- the k-means math is
+ * unchanged, only the execution is reorganised (same abstract; the Japanese
+ * Hacker News summary, section "what Flash-KMeans changes"):
+ *   - FlashAssign fuses the distance computation with an online argmin, so the
+ *     N x K distance matrix is never written to HBM;
+ *   - the sort-inverse update groups points by cluster id (an inverse map with
+ *     segment offsets) and sums each segment locally instead of scattering
+ *     atomics into the centroid sums;
+ *   - chunked-stream overlap streams inputs larger than device memory from the
+ *     host, overlapping the copy of one chunk with the compute of another.
+ *
+ * Conventions shared by every entry point
+ *   Layout     X is row-major N x D (batched: B x N x D, problem-major);
+ *              centroids K x D (batched B x K x D); labels N (B x N) int32;
+ *              everything contiguous, no strides.
+ *   dtype      FK_F32, FK_F16 or FK_BF16 tags the element type of X (and of C
+ *              where C is given in the input type).  Arithmetic accumulates in
+ *              fp32.  fp16/bf16 assignment runs on tcgen05 tensor cores when
+ *              D is a multiple of 8 and 8 <= D <= 128; every other case runs on
+ *              a CUDA-core kernel (fp32 always does).
+ *   Distances  label[i] = argmin_k |x_i - c_k|^2 with ties to the LOWEST k
+ *              (the pages are silent on ties).  mindist[i] = that squared
+ *              distance, clamped at 0.  The tensor path evaluates
+ *              |c|^2 - 2<x,c> (+|x|^2 for mindist) in fp32.
+ *   Update     C_k = mean of the points with label k, in fp32; a cluster
+ *              that receives no point keeps its previous centroid and gets
+ *              count 0 (the pages are silent on empty clusters).
+ *   Memory     Pointers documented as "device" must be device memory of the
+ *              current CUDA device; "host" means host memory (pinned memory
+ *              gives asynchronous copies, pageable memory still works).  All
+ *              device arrays are owned by the caller.  The library keeps a
+ *              per-(device, stream) scratch cache that it grows on demand with
+ *              stream-ordered allocation; fk_release_workspace() returns it.
+ *              Device pointers to X and C must be 16-byte aligned for the
+ *              tensor-core path (else the CUDA-core kernel is used).
+ *   Streams    stream is a cudaStream_t (NULL = legacy default stream).
+ *              fk_assign / fk_update and their batched forms only enqueue work
+ *              and return; fk_lloyd* and fk_lloyd_ooc synchronise the stream
+ *              before returning.  Calls that share a device and a stream are
+ *              ordered; concurrent calls on different streams use separate
+ *              scratch.
+ *   Errors     Every entry point returns an fk_status.  Argument errors are
+ *              detected on the host before any work is enqueued (nothing is
+ *              written).  Errors found on the device (a label outside [0, K)
+ *              given to fk_update, a wait that ran out of time) are recorded in
+ *              a per-device status word that fk_sync() returns and clears;
+ *              the synchronous entry points return it themselves.
+ *              fk_last_error_message() describes the last non-OK status of
+ *              the calling thread.
+ *   Limits     1 <= D <= 1024; 1 <= K <= 2^22 (B*K <= 2^22); 1 <= B <= 65535;
+ *              0 <= N, B*N < 2^31; K <= N is NOT required.
+ */
+#ifndef FK_H_
+#define FK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FK_API __attribute__((visibility("default")))
+#else
+#define FK_API
+#endif
+
+typedef struct CUstream_st *fk_stream_t; /* identical to cudaStream_t */
+
+typedef enum { FK_F32 = 0, FK_F16 = 1, FK_BF16 = 2 } fk_dtype;
+
+typedef int fk_status;
+enum {
+  FK_OK = 0,
+  FK_ERR_INVALID_ARG = -1, /* bad pointer, size or dtype                       */
+  FK_ERR_UNSUPPORTED = -2, /* valid request this build cannot run              */
+  FK_ERR_CUDA = -3,        /* a CUDA runtime call failed (no device, launch)   */
+  FK_ERR_OOM = -4,         /* device or pinned allocation failed               */
+  FK_ERR_TIMEOUT = -5,     /* a device-side wait exceeded its time limit       */
+  FK_ERR_HOST_IO = -6,     /* a host<->device copy failed (out-of-core path)   */
+  FK_ERR_BAD_LABEL = -7    /* fk_update saw a label outside [0, K)             */
+};
+
+/* ------------------------------------------------------------------------
+ * fk_assign -- assignment stage (FlashAssign).
+ *   Flash-KMeans abstract: FlashAssign computes each distance and folds it
+ *   into a running argmin on chip, so the N x K distances are never stored.
+ *   X        device, N x D, dtype dt
+ *   C        device, K x D, dtype dt (centroids already in the input type)
+ *   labels   device, N int32 (out)
+ *   mindist  device, N fp32 (out) or NULL
+ *   N may be 0 (nothing is launched).
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K,
+                    int32_t *labels, float *mindist, fk_stream_t stream);
+
+/* fk_assign_batched -- B independent assignment problems in one launch.
+ *   X B x N x D, C B x K x D, labels B x N, mindist B x N or NULL (device).
+ *   Problem b compares rows of X[b] only with centroids of C[b]; labels are
+ *   in [0, K) within each problem. */
+FK_API fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C,
+                            int K, int32_t *labels, float *mindist, fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Two-phase assignment for callers that iterate (Lloyd loops, benchmarks).
+ *
+ * fk_norms_len -- number of floats of the norm buffer for B problems of K
+ *   centroids (K rounded up to the 256-centroid tile, per problem).
+ * fk_prepare_centroids -- the preparation step of the assignment stage:
+ *   C_dt = C32 rounded to dt (round-to-nearest-even; a plain copy for
+ *   FK_F32, skipped when C_dt == C32) and norms = |C_dt[k]|^2 in fp32, with
+ *   +inf in the padding so padded columns never win.  One kernel.
+ *   C32 device B x K x D fp32; C_dt device B x K x D of dt; norms device
+ *   fk_norms_len(B, K) floats.
+ * fk_assign_prepared -- fk_assign_batched against prepared centroids and
+ *   norms; launches exactly one kernel (the CUDA-core kernel, which computes
+ *   direct differences, does not read the norms).
+ * ------------------------------------------------------------------------ */
+FK_API int64_t fk_norms_len(int B, int K);
+FK_API fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt,
+                                      float *norms, fk_stream_t stream);
+FK_API fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt,
+                                    int K, const float *norms, int32_t *labels, float *mindist,
+                                    fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fk_update -- centroid-update stage (sort-inverse update).
+ *   Flash-KMeans abstract: the update builds an explicit inverse map from
+ *   clusters to their points and sums each cluster's segment locally instead
+ *   of scattering contended atomics.  Here: a stable radix sort of the labels gives the inverse
+ *   map (point ids grouped by cluster) and segment offsets; each segment is
+ *   summed in fp32 by contention-free reductions, partial sums of segments
+ *   that cross work-chunk borders are combined in a fixed order (the result is
+ *   deterministic), and divided by the count.
+ *   X        device, N x D, dtype dt
+ *   labels   device, N int32, each in [0, K)
+ *   C        device, K x D fp32, in: previous centroids, out: new centroids
+ *            (rows of empty clusters are left untouched)
+ *   counts   device, K int32 (out) or NULL
+ *   A label outside [0, K) is counted in cluster 0 and reported as
+ *   FK_ERR_BAD_LABEL by fk_sync().
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_update(const void *X, const int32_t *labels, int64_t N, int D, fk_dtype dt, int K,
+                    float *C, int32_t *counts, fk_stream_t stream);
+
+/* fk_update_batched -- B independent update problems (labels B x N, C B x K
+ * x D fp32 in/out, counts B x K or NULL), one sort over B*K segments. */
+FK_API fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t N, int D,
+                            fk_dtype dt, int K, float *C, int32_t *counts, fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fk_lloyd -- `iters` Lloyd iterations, device resident.
+ *   Iteration t assigns X against C_t rounded (round-to-nearest-even) to the
+ *   input type (fp16/bf16; fp32 uses C_t as is), then sets C_{t+1} = the
+ *   cluster means in fp32.  On return C holds C_iters, labels the last
+ *   assignment (made against C_{iters-1}), mindist (or NULL) its squared
+ *   distances and counts (or NULL) its cluster sizes.  iters >= 1.
+ *   X device N x D; C device K x D fp32 in/out; labels device N int32.
+ *   Synchronises `stream`; returns the first device-side error, if any.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_lloyd(const void *X, int64_t N, int D, fk_dtype dt, float *C, int K,
+                   int32_t *labels, float *mindist, int32_t *counts, int iters,
+                   fk_stream_t stream);
+
+/* fk_lloyd_batched -- fk_lloyd over B independent problems in one launch per
+ * stage (shapes as in fk_assign_batched / fk_update_batched). */
+FK_API fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, float *C, int K,
+                           int32_t *labels, float *mindist, int32_t *counts, int iters,
+                           fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fk_lloyd_ooc -- out-of-core Lloyd with chunked-stream overlap.
+ *   Flash-KMeans abstract ("chunked-stream overlap"); the Japanese summary
+ *   adds that PCIe transfers overlap compute when the input exceeds VRAM.
+ *   X_host stays in host memory: every iteration streams it in chunks of
+ *   chunk_rows rows through a ring of device buffers; the copy of chunk c+1
+ *   runs on a side stream while chunk c is assigned and its per-cluster sums
+ *   are accumulated (fp64 accumulators, no atomics).  The iteration ends by
+ *   dividing.  The result equals fk_lloyd on the same data up to the
+ *   summation order of the means.
+ *   X_host       host, N x D dtype dt (pinned for overlap)
+ *   C_host       host, K x D fp32, in/out
+ *   labels_host  host, N int32 (out, last iteration) or NULL
+ *   counts_host  host, K int32 (out) or NULL
+ *   chunk_rows   rows per chunk, >= 1 (clamped to N); the library allocates
+ *                2 chunk buffers plus per-chunk scratch and frees them before
+ *                returning.
+ *   Synchronous: returns when C_host (and labels/counts) are written.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float *C_host, int K,
+                       int32_t *labels_host, int32_t *counts_host, int iters, int64_t chunk_rows,
+                       fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status, diagnostics and control.
+ * ------------------------------------------------------------------------ */
+
+/* Synchronise `stream`, then return and clear the current device's status
+ * word (FK_ERR_BAD_LABEL, FK_ERR_TIMEOUT) or a CUDA error; FK_OK otherwise. */
+FK_API fk_status fk_sync(fk_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+FK_API const char *fk_status_string(fk_status s);
+
+/* Last non-OK status returned to the calling thread (FK_OK if none), and a
+ * human-readable message for it.  Reading does not clear it. */
+FK_API fk_status fk_get_last_error(void);
+FK_API const char *fk_last_error_message(void);
+
+/* Number of kernels this library has launched in this process (all devices). */
+FK_API uint64_t fk_launch_count(void);
+
+/* Which assignment kernel fk_assign would run for this request:
+ * 1 = tcgen05 tensor-core kernel, 2 = CUDA-core kernel, or a negative status
+ * for an invalid request.  Host-only: queries no device. */
+FK_API int fk_assign_path(int64_t N, int D, fk_dtype dt, int K, int B);
+
+/* Force the assignment kernel: 0 = automatic (default), 1 = tensor-core
+ * (requests it cannot serve fail with FK_ERR_UNSUPPORTED), 2 = CUDA-core.
+ * Process-wide; used by tests to compare the two kernels on one input. */
+FK_API fk_status fk_set_assign_path(int path);
+
+/* Time limit of every device-side wait loop, in nanoseconds (default 2e9).
+ * A wait that exceeds it makes the kernel stop, release what it holds and
+ * record FK_ERR_TIMEOUT.  0 restores the default. */
+FK_API fk_status fk_set_wait_timeout_ns(uint64_t ns);
+
+/* Self-test of the wait-timeout mechanism: runs one small kernel that waits
+ * on a shared-memory barrier nothing will complete, bounded by `ns`; returns
+ * the status the kernel recorded (FK_ERR_TIMEOUT when the mechanism works).
+ * Synchronises `stream`. */
+FK_API fk_status fk_debug_wait_timeout(uint64_t ns, fk_stream_t stream);
+
+/* Free the scratch cached for the current device (all streams).  The caller
+ * must ensure no fk_* work is still running on that device. */
+FK_API fk_status fk_release_workspace(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+FK_API int fk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FK_H_ */

@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Small and ragged shapes span several tiles of every kernel (256-point units,
+256-centroid tiles, 4096-key sort tiles, chunked segment sums) and their
+tails; inputs come from the seeded generators only."""
+import numpy as np
+import pytest
+import torch
+
+import distance_argmin_flashassign_b200 as fk
+import oracle
+import workloads
+from tests.parity import TORCH_DT, check_centroids, check_labels, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def mixture(N, D, K, dtype, seed=0, cfg="tiny_f32", n_centers=None):
+    s = workloads.spec(cfg, N=N, D=D, K=K, dtype=dtype, n_centers=n_centers or max(K, 2), B=1)
+    w = workloads.make(s, seed=seed)
+    return w.X, w.C0
+
+
+def c_in(C0, dtype):
+    return C0.to(TORCH_DT[dtype])
+
+
+ASSIGN_SHAPES = [  # (N, D, K): tails in N, D and K; tensor and CUDA-core paths
+    (1000, 32, 10), (3001, 128, 300), (257, 8, 1), (5000, 64, 1024), (600, 100, 37),
+    (2000, 120, 513), (1000, 16, 700), (4097, 128, 2048), (700, 40, 256), (300, 128, 1),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("shape", ASSIGN_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_assign_matches_oracle(shape, dtype):
+    N, D, K = shape
+    X, C0 = mixture(N, D, K, dtype, seed=N + D + K)
+    C = c_in(C0, dtype)
+    Xd, Cd = X.to(DEV), C.to(DEV)
+    labels, mind = fk.fk_assign(Xd, Cd, want_mindist=True)
+    fk.fk_sync()
+    check_labels(f64(X), f64(C), labels, dtype, gpu_mindist=mind)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_tensor_and_cuda_core_paths_agree(dtype):
+    X, C0 = mixture(6000, 128, 777, dtype, seed=3)
+    Xd, Cd = X.to(DEV), c_in(C0, dtype).to(DEV)
+    try:
+        fk.fk_set_assign_path(1)
+        l1, m1 = fk.fk_assign(Xd, Cd, want_mindist=True)
+        fk.fk_set_assign_path(2)
+        l2, m2 = fk.fk_assign(Xd, Cd, want_mindist=True)
+        fk.fk_sync()
+    finally:
+        fk.fk_set_assign_path(0)
+    check_labels(f64(X), f64(Cd), l1, dtype, gpu_mindist=m1)
+    check_labels(f64(X), f64(Cd), l2, dtype, gpu_mindist=m2)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("path", [1, 2])
+def test_integer_inputs_bit_exact_with_ties(dtype, path):
+    """Small integers: products and fp32 sums are exact, so labels (including
+    lowest-index tie-breaks on duplicated centroids) and mindist are exact."""
+    if dtype == "f32" and path == 1:
+        pytest.skip("fp32 runs on the CUDA-core kernel only")
+    g = torch.Generator().manual_seed(5)
+    N, D, K = 3000, 64, 300
+    X = torch.randint(-8, 9, (N, D), generator=g).to(TORCH_DT[dtype])
+    C = torch.cat([X[:100], X[:100], torch.randint(-8, 9, (100, D), generator=g).to(TORCH_DT[dtype])])
+    C[250] = C[10]  # later duplicate of an earlier centroid
+    try:
+        fk.fk_set_assign_path(path)
+        labels, mind = fk.fk_assign(X.to(DEV), C.to(DEV), want_mindist=True)
+        fk.fk_sync()
+    finally:
+        fk.fk_set_assign_path(0)
+    lab, md, _ = oracle.assign(f64(X), f64(C))
+    assert np.array_equal(labels.cpu().numpy(), lab)
+    assert np.array_equal(mind.cpu().numpy().astype(np.float64), md)
+    assert labels[:100].cpu().tolist() == list(range(100))
+
+
+def test_assign_batched_matches_per_problem():
+    B, N, D, K = 5, 1500, 128, 300
+    s = workloads.spec("batched_bf16", N=N, K=K, n_centers=64, B=B)
+    w = workloads.make(s, seed=1)
+    X, C = w.X, w.C0.to(torch.bfloat16)
+    labels, mind = fk.fk_assign(X.to(DEV), C.to(DEV), want_mindist=True)
+    fk.fk_sync()
+    for b in range(B):
+        check_labels(f64(X[b]), f64(C[b]), labels[b], "bf16", gpu_mindist=mind[b])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("kind", ["uniform", "zipf", "one", "sparse"])
+@pytest.mark.parametrize("ND", [(5000, 128, 300), (20000, 32, 2100), (3000, 100, 17), (9000, 8, 64), (100, 1, 300)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_update_matches_oracle(ND, kind, dtype):
+    N, D, K = ND
+    X, _ = mixture(N, D, 2, dtype, seed=N + K)
+    labels = workloads.labels(N, K, seed=K, kind=kind)
+    C_prev = workloads.perturb(torch.zeros(K, D), 1.0, seed=D)
+    C = C_prev.clone().to(DEV)
+    counts = torch.empty(K, dtype=torch.int32, device=DEV)
+    fk.fk_update(X.to(DEV), labels.to(DEV), C, counts)
+    fk.fk_sync()
+    Cn, cnt = oracle.update(f64(X), labels.numpy(), K, f64(C_prev))
+    assert np.array_equal(counts.cpu().numpy(), cnt)
+    empty = cnt == 0
+    assert torch.equal(C.cpu()[torch.from_numpy(empty)], C_prev[torch.from_numpy(empty)])
+    check_centroids(C, Cn)
+
+
+def test_update_is_deterministic():
+    X, _ = mixture(50000, 128, 2, "bf16", seed=9)
+    labels = workloads.labels(50000, 1000, kind="zipf").to(DEV)
+    Xd = X.to(DEV)
+    outs = []
+    for _ in range(2):
+        C = torch.zeros(1000, 128, device=DEV)
+        fk.fk_update(Xd, labels, C)
+        outs.append(C.clone())
+    fk.fk_sync()
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_update_batched():
+    B, N, D, K = 4, 3000, 64, 500
+    s = workloads.spec("batched_bf16", N=N, D=D, K=K, n_centers=50, B=B)
+    X = workloads.make(s, seed=2).X
+    labels = torch.stack([workloads.labels(N, K, seed=b, kind="zipf") for b in range(B)])
+    C = torch.zeros(B, K, D, device=DEV)
+    counts = torch.empty(B, K, dtype=torch.int32, device=DEV)
+    fk.fk_update(X.to(DEV), labels.to(DEV), C, counts)
+    fk.fk_sync()
+    for b in range(B):
+        Cn, cnt = oracle.update(f64(X[b]), labels[b].numpy(), K, np.zeros((K, D)))
+        assert np.array_equal(counts[b].cpu().numpy(), cnt)
+        check_centroids(C[b], Cn)
+
+
+def test_update_reports_bad_label():
+    X = torch.randn(1000, 32, device=DEV)
+    labels = torch.zeros(1000, dtype=torch.int32, device=DEV)
+    labels[17] = 40
+    C = torch.zeros(8, 32, device=DEV)
+    fk.fk_update(X, labels, C)
+    with pytest.raises(fk.FKError) as e:
+        fk.fk_sync()
+    assert e.value.status == fk.FK_ERR_BAD_LABEL
+    fk.fk_sync()  # the status word was cleared
+
+
+@pytest.mark.parametrize("cfg,N,K,iters,nc", [
+    ("tiny_f32", 32768, 128, 5, 128),          # the tiny workload at full size
+    ("embed_f16", 16384, 256, 3, 256),
+    ("zipf_bf16", 16384, 1024, 2, 1024),
+])
+def test_lloyd_matches_oracle(cfg, N, K, iters, nc):
+    s = workloads.spec(cfg, N=N, K=K, n_centers=nc)
+    w = workloads.make(s, seed=0)
+    C = w.C0.clone().to(DEV)
+    C, labels, mind, counts = fk.fk_lloyd(w.X.to(DEV), C, iters, want_mindist=True)
+    out = oracle.lloyd(f64(w.X), f64(w.C0), iters, s.dtype)
+    check_centroids(C, out["C"])
+    # the last assignment was made against C_{iters-1}: rebuild it from the oracle trajectory
+    Cprev = oracle.lloyd(f64(w.X), f64(w.C0), iters - 1, s.dtype)["C"] if iters > 1 else f64(w.C0)
+    check_labels(f64(w.X), oracle.round_to(s.dtype, Cprev), labels, s.dtype, gpu_mindist=mind)
+    assert int(counts.sum()) == N
+    assert torch.equal(counts.cpu().long(), torch.bincount(labels.cpu().long(), minlength=K))
+
+
+def test_lloyd_batched_matches_oracle():
+    s = workloads.spec("batched_bf16", N=4096, K=256, n_centers=256, B=3)
+    w = workloads.make(s, seed=0)
+    C = w.C0.clone().to(DEV)
+    C, labels, _, counts = fk.fk_lloyd(w.X.to(DEV), C, 3)
+    for b in range(3):
+        out = oracle.lloyd(f64(w.X[b]), f64(w.C0[b]), 3, "bf16")
+        check_centroids(C[b], out["C"])
+        assert int(counts[b].sum()) == 4096
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_ooc_matches_in_core(dtype):
+    N, D, K = 50001, 128 if dtype == "f16" else 32, 300
+    cfg = "ooc_f16" if dtype == "f16" else "tiny_f32"
+    s = workloads.spec(cfg, N=N, D=D, K=K, n_centers=K, dtype=dtype)
+    w = workloads.make(s, seed=4)
+    Xh = w.X.pin_memory()
+    Ch = w.C0.clone()
+    lab_h = torch.empty(N, dtype=torch.int32).pin_memory()
+    cnt_h = torch.empty(K, dtype=torch.int32)
+    fk.fk_lloyd_ooc(Xh, Ch, 2, 12345, lab_h, cnt_h)
+    Cd = w.C0.clone().to(DEV)
+    Cd, labels, _, counts = fk.fk_lloyd(w.X.to(DEV), Cd, 2)
+    assert rel_l2(Ch.numpy(), f64(Cd)) <= 1e-5
+    mism = int((lab_h != labels.cpu()).sum())
+    assert mism <= 1e-4 * N
+    out = oracle.lloyd(f64(w.X), f64(w.C0), 2, dtype)
+    check_centroids(Ch, out["C"])
+    assert int(cnt_h.sum()) == N
+
+
+def test_edge_cases():
+    # K = 1: every label 0, centroid = mean
+    X = torch.randn(777, 16, device=DEV, dtype=torch.float16)
+    C = X[:1].float().clone()
+    C, labels, _, counts = fk.fk_lloyd(X, C, 1)
+    assert int(labels.abs().sum()) == 0 and counts.tolist() == [777]
+    np.testing.assert_allclose(C.cpu().numpy()[0], f64(X).mean(0), rtol=1e-3, atol=1e-3)
+    # K > N: empty clusters keep their centroid
+    X = torch.randn(50, 24, device=DEV)
+    C0 = torch.randn(300, 24, device=DEV)
+    C = C0.clone()
+    C, labels, _, counts = fk.fk_lloyd(X, C, 1)
+    empty = counts == 0
+    assert int(empty.sum()) >= 250 and torch.equal(C[empty], C0[empty])
+    # N = 0: no-op
+    lab = torch.empty(0, dtype=torch.int32, device=DEV)
+    fk.fk_assign(torch.empty(0, 8, device=DEV, dtype=torch.float16), torch.zeros(3, 8, device=DEV,
+                 dtype=torch.float16), labels=lab)
+    # D = 1 and identical points
+    X = torch.full((1000, 1), 2.5, device=DEV)
+    labels, mind = fk.fk_assign(X, torch.tensor([[1.0], [4.0], [2.5], [2.5]], device=DEV), want_mindist=True)
+    fk.fk_sync()
+    assert torch.all(labels == 2) and torch.all(mind == 0)
+
+
+def test_wait_timeout_mechanism_and_recovery():
+    assert fk.fk_debug_wait_timeout(1_000_000) == fk.FK_ERR_TIMEOUT
+    X = torch.randn(1000, 64, device=DEV, dtype=torch.float16)
+    labels, _ = fk.fk_assign(X, X[:10].clone())
+    fk.fk_sync()
+    assert labels[:10].cpu().tolist() == list(range(10))
+
+
+def test_launch_counter_counts_kernels():
+    X = torch.randn(5000, 128, device=DEV, dtype=torch.float16)
+    n0 = fk.fk_launch_count()
+    fk.fk_assign(X, X[:300].clone())
+    fk.fk_sync()
+    assert fk.fk_launch_count() - n0 == 2  # norms + tensor-core assign
