@@ -4,7 +4,7 @@ One step = one pass of the whole hot path on the embedding workload
 (N = 1,048,576 points, D = 128, fp16, K = 1,024 centroids; the workload the
 headline metric is quoted on):
 
-    fk_prepare_centroids  (round fp32 centroids to fp16, centroid norms)
+    fk_prepare_centroids  (round fp32 centroids to fp16, bias -|c|^2/2)
     fk_assign_prepared    (tcgen05 FlashAssign: distances + online argmin)
     fk_update             (sort-inverse update: radix sort, segment offsets,
                            segmented sums, divide)
@@ -220,16 +220,16 @@ def bench_gpu(args):
     X = w.X
     B, N, D, K = s.B, s.N, s.D, s.K
     C = w.C0.clone()
-    C_dt, norms = fk.fk_prepare_centroids(C, dt)
+    C_dt, bias = fk.fk_prepare_centroids(C, dt)
     labels = torch.empty(((B, N) if B > 1 else (N,)), dtype=torch.int32, device=dev)
     counts = torch.empty(((B, K) if B > 1 else (K,)), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
-        fk.fk_prepare_centroids(C, dt, C_dt, norms)
+        fk.fk_prepare_centroids(C, dt, C_dt, bias)
         if ev:
             ev[0].record(stream)
-        fk.fk_assign_prepared(X, C_dt, norms, labels)
+        fk.fk_assign_prepared(X, C_dt, bias, labels)
         if ev:
             ev[1].record(stream)
         fk.fk_update(X, labels, C, counts)

@@ -53,7 +53,7 @@ def _load():
         "fk_lloyd": [V, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_batched": [V, I, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_ooc": [V, I64, I, I, V, I, V, V, I, I64, V],
-        "fk_norms_len": [I, I],
+        "fk_bias_len": [I, I],
         "fk_prepare_centroids": [V, I, I, I, I, V, V, V],
         "fk_assign_prepared": [V, I, I64, I, I, V, I, V, V, V, V],
         "fk_sync": [V],
@@ -75,14 +75,14 @@ def _load():
     lib.fk_status_string.restype = ctypes.c_char_p
     lib.fk_last_error_message.restype = ctypes.c_char_p
     lib.fk_launch_count.restype = ctypes.c_uint64
-    lib.fk_norms_len.restype = ctypes.c_int64
+    lib.fk_bias_len.restype = ctypes.c_int64
     return lib
 
 
 lib = _load()
 
 # names declared in include/fk.h (the C ABI this binding mirrors)
-ABI_NAMES = ("fk_norms_len", "fk_prepare_centroids", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_lloyd",
+ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_lloyd",
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_version")
@@ -148,28 +148,28 @@ def fk_assign(X, C, labels=None, mindist=None, want_mindist=False, stream=None):
     return labels, mindist
 
 
-def fk_prepare_centroids(C, dtype, C_dt=None, norms=None, stream=None):
-    """Round fp32 centroids (K x D or B x K x D) to ``dtype`` and compute their
-    padded squared norms.  Returns (C_dt, norms)."""
+def fk_prepare_centroids(C, dtype, C_dt=None, bias=None, stream=None):
+    """Round fp32 centroids (K x D or B x K x D) to ``dtype`` and compute the
+    padded bias -|c|^2/2.  Returns (C_dt, bias)."""
     bat = C.dim() == 3
     B, K, D = (C.shape if bat else (1,) + tuple(C.shape))
     _need(C, "C", torch.float32, C.shape, C.device)
     if C_dt is None:
         C_dt = C if dtype == torch.float32 else torch.empty(C.shape, dtype=dtype, device=C.device)
     _need(C_dt, "C_dt", dtype, C.shape, C.device)
-    n = int(lib.fk_norms_len(B, K))
-    if norms is None:
-        norms = torch.empty(n, dtype=torch.float32, device=C.device)
-    _need(norms, "norms", torch.float32, (n,), C.device)
-    _check(lib.fk_prepare_centroids(_ptr(C), B, K, D, _DT[dtype], _ptr(C_dt), _ptr(norms), _stream(stream)))
-    return C_dt, norms
+    n = int(lib.fk_bias_len(B, K))
+    if bias is None:
+        bias = torch.empty(n, dtype=torch.float32, device=C.device)
+    _need(bias, "bias", torch.float32, (n,), C.device)
+    _check(lib.fk_prepare_centroids(_ptr(C), B, K, D, _DT[dtype], _ptr(C_dt), _ptr(bias), _stream(stream)))
+    return C_dt, bias
 
 
-def fk_assign_prepared(X, C_dt, norms, labels, mindist=None, stream=None):
+def fk_assign_prepared(X, C_dt, bias, labels, mindist=None, stream=None):
     """One-kernel assignment against the output of ``fk_prepare_centroids``."""
     B, N, D, bat = _dims(X)
     K = C_dt.shape[-2]
-    _check(lib.fk_assign_prepared(_ptr(X), B, N, D, _dtype(X), _ptr(C_dt), K, _ptr(norms), _ptr(labels),
+    _check(lib.fk_assign_prepared(_ptr(X), B, N, D, _dtype(X), _ptr(C_dt), K, _ptr(bias), _ptr(labels),
                                   _ptr(mindist), _stream(stream)))
     return labels, mindist
 

@@ -11,16 +11,27 @@
 //     a ring of shared-memory stages (128-byte swizzle, one 64-element k-block
 //     per stage);
 //   * one thread issues tcgen05.mma (M=128, N=256, K=16, fp32 accumulate)
-//     into two TMEM accumulators of 128 x 256 fp32, one per sub-tile;
-//   * eight epilogue warps drain each accumulator with tcgen05.ld, form
-//     |c|^2 - 2<x,c> with one FMA per element and keep a running
-//     (min, argmin) per point in registers; ties keep the lower index
-//     because columns are scanned in ascending order with a strict "<".
-//     Warpgroup 0 scans columns [0,128) of every tile, warpgroup 1 [128,256);
-//     the two halves are merged at the end of the unit.
+//     into two TMEM accumulators of 128 x 256 fp32, one per sub-tile.  Each
+//     accumulator already holds the bias -|c|^2/2 of its columns when the MMA
+//     starts, so it ends holding the score s = <x,c> - |c|^2/2, whose arg-max
+//     is the arg-min of |x - c|^2: no per-distance arithmetic is left for the
+//     epilogue but the arg-max itself;
+//   * four epilogue warpgroups drain the accumulators with tcgen05.ld:
+//     warpgroups 0-1 own sub-tile 0, 2-3 own sub-tile 1, and within a pair
+//     one scans columns [0,128) of every tile and the other [128,256).  Each
+//     thread owns one point (TMEM lane == row).  Per 32-column chunk a
+//     3-input-max tree (half an ALU op per score; the ALU pipe runs at half
+//     rate and bounds this epilogue) gives the chunk maximum; when it beats
+//     the point's running maximum (strict ">", so an earlier column keeps a
+//     tie) the lane copies the chunk into a register-resident candidate.  The
+//     lowest column of the candidate holding the maximum is found once per
+//     unit.  After reading a chunk the thread writes the next tile's bias
+//     into the same TMEM columns (tcgen05.st), re-arming the accumulator.
+//     The two column halves of a point are merged at the end of the unit
+//     (score, then lower index).
 //
-// Only labels (and optionally |x|^2 + min) leave the chip.  X, C and the
-// centroid norms are read; nothing else is written.
+// Only labels (and optionally |x|^2 - 2 max s) leave the chip.  X, C and the
+// bias are read; nothing else is written.
 //
 // Every wait is an mbarrier wait bounded in time; on expiry the CTA records
 // FK_ERR_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
@@ -39,9 +50,10 @@ constexpr int kTileN = 256;                // centroids per tile (MMA N)
 constexpr int kBlkK = 64;                  // elements per k-block (128 bytes)
 constexpr int kSubBytes = kRowsSub * 128;  // one sub-tile k-block, 16 KB
 constexpr int kStageBytes = kTileN * 128;  // one centroid k-block, 32 KB
-constexpr int kEpiWarps = 8;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 32 * 10;
+constexpr int kEpiWarps = 16;                 // four epilogue warpgroups
+constexpr int kAccWarps = 8;                  // warps draining one accumulator
+constexpr int kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kThreads = 32 * 18;
 constexpr uint32_t kTmemCols = 512;        // two 256-column fp32 accumulators
 
 template <int KB> struct TcCfg {
@@ -57,12 +69,31 @@ template <int KB> struct TcCfg {
   static_assert(NST >= KB, "a whole centroid tile must fit in the stage ring");
 };
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 32 consecutive bias values (uniform address across the warp, L1 cached).
+__device__ __forceinline__ void load_bias32(const float *p, uint32_t (&w)[32]) {
+  const float4 *p4 = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float4 t = __ldg(p4 + e);
+    w[4 * e] = __float_as_uint(t.x);
+    w[4 * e + 1] = __float_as_uint(t.y);
+    w[4 * e + 2] = __float_as_uint(t.z);
+    w[4 * e + 3] = __float_as_uint(t.w);
+  }
+}
+
 struct TcParams {
   int N, K, Kpad, ntiles, upb, total_units;
   uint32_t idesc;
   int is_bf16;
   uint32_t dyn_bytes;
-  const float *cn;
+  const float *bias;  // -|c|^2/2 per centroid, -inf in the padding
   int32_t *labels;
   float *mindist;
   DevCtl ctl;
@@ -113,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(accfull(g), 1);
-      mbar_init(accempty(g), kEpiWarps);
+      mbar_init(accempty(g), kAccWarps);
     }
     mbar_init(xchg_full, kEpiWarps);
     mbar_init(xchg_empty, kEpiWarps);
@@ -186,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           tc_fence_after();
-          if (!(ok = mbar_wait(accempty(0), ae0 ^ 1u, abort_flag, p.ctl))) break;
+          if (!(ok = mbar_wait(accempty(0), ae0, abort_flag, p.ctl))) break;
           ae0 ^= 1u;
           tc_fence_after();
 #pragma unroll
@@ -195,10 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = desc_kmajor_sw128(sC + stg[kb] * kStageBytes);
 #pragma unroll
             for (int k = 0; k < kBlkK / 16; ++k)
-              tc_mma_f16(tbase, ad + 2 * k, bd + 2 * k, p.idesc, (kb | k) != 0);
+              tc_mma_f16(tbase, ad + 2 * k, bd + 2 * k, p.idesc, 1u);
           }
           tc_commit(accfull(0));
-          if (!(ok = mbar_wait(accempty(1), ae1 ^ 1u, abort_flag, p.ctl))) break;
+          if (!(ok = mbar_wait(accempty(1), ae1, abort_flag, p.ctl))) break;
           ae1 ^= 1u;
           tc_fence_after();
 #pragma unroll
@@ -207,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = desc_kmajor_sw128(sC + stg[kb] * kStageBytes);
 #pragma unroll
             for (int k = 0; k < kBlkK / 16; ++k)
-              tc_mma_f16(tbase + kTileN, ad + 2 * k, bd + 2 * k, p.idesc, (kb | k) != 0);
+              tc_mma_f16(tbase + kTileN, ad + 2 * k, bd + 2 * k, p.idesc, 1u);
           }
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) tc_commit(empty(stg[kb]));
@@ -224,29 +255,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------ epilogue ----
     const int wg = warp >> 2, q = warp & 3;
+    const int g = wg >> 1;     // sub-tile (accumulator) of this warpgroup
+    const int h = wg & 1;      // column half of every tile
     const int r = q * 32 + lane;  // row within the sub-tile == TMEM lane
-    const uint32_t t_row = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(wg * 128);
-    uint32_t xb = 0, xph = 0, af0 = 0, af1 = 0, xc = 0;
+    const uint32_t t_row = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * kTileN + h * 128);
+    const uint32_t my_full = accfull(g), my_empty = accempty(g);
+    // bias of tile j of the unit u, for this warpgroup's 128 columns
+    auto bias_of = [&](int u, int j) {
+      return p.bias + (size_t)(u / p.upb) * p.Kpad + j * kTileN + h * 128;
+    };
+    // Every accumulator starts each tile holding the bias: the first tile's
+    // now, every later tile's while the previous tile is drained.
+    if ((int)blockIdx.x < p.total_units) {
+      const float *bp = bias_of(blockIdx.x, 0);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[32];
+        load_bias32(bp + c * 32, w);
+        FK_TMEM_ST32(t_row + c * 32, w);
+      }
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(my_empty);
+
+    uint32_t xb = 0, xph = 0, af = 0, xc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x, xc ^= 1u) {
       const int b = u / p.upb, r0 = (u % p.upb) * kRowsUnit;
       if (!(ok = mbar_wait(xfull(xb), xph, abort_flag, p.ctl))) break;
       float xn = 0.f;
-      if (p.mindist) {  // |x|^2 of row r of sub-tile wg, from the swizzled tile
+      if (p.mindist && h == 0) {  // |x|^2 of row r of sub-tile g, from the swizzled tile
         for (int kb = 0; kb < KB; ++kb) {
-          const uint8_t *rowp = sm + ((xb * kSubs + wg) * KB + kb) * kSubBytes + r * 128;
+          const uint8_t *rowp = sm + ((xb * kSubs + g) * KB + kb) * kSubBytes + r * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 w = *reinterpret_cast<const uint4 *>(rowp + ((c ^ (r & 7)) << 4));
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
+            for (int e = 0; e < 4; ++e) {
               float lo, hi;
               if (p.is_bf16) {
-                lo = __uint_as_float(ws[h] << 16);
-                hi = __uint_as_float(ws[h] & 0xffff0000u);
+                lo = __uint_as_float(ws[e] << 16);
+                hi = __uint_as_float(ws[e] & 0xffff0000u);
               } else {
-                const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[h]);
+                const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[e]);
                 lo = __low2float(h2);
                 hi = __high2float(h2);
               }
@@ -260,67 +314,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(xempty(xb));
       if (++xb == XBUF) { xb = 0; xph ^= 1u; }
 
-      float best[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
-      int bidx[2] = {0, 0};
+      // score s = <x,c> - |c|^2/2 (argmax s == argmin |x-c|^2); running max and
+      // the 32-column chunk that first reached it
+      float cbest = __int_as_float(0xff800000);
+      int cbase = 0;
+      uint32_t cand[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) cand[t] = 0u;
       for (int j = 0; ok && j < p.ntiles; ++j) {
-        const int col0 = j * kTileN + wg * 128;
-        const float4 *cn4 = reinterpret_cast<const float4 *>(p.cn + (size_t)b * p.Kpad + col0);
-#pragma unroll
-        for (int g = 0; g < kSubs; ++g) {
-          if (!(ok = mbar_wait(accfull(g), g ? af1 : af0, abort_flag, p.ctl))) break;
-          if (g) af1 ^= 1u; else af0 ^= 1u;
-          tc_fence_after();
-          float cb = best[g];
-          int bi = bidx[g];
+        const int col0 = j * kTileN + h * 128;
+        int nu = u, nj = j + 1;  // the tile this accumulator holds next
+        if (nj == p.ntiles) { nu = u + gridDim.x; nj = 0; }
+        const float *nbp = nu < p.total_units ? bias_of(nu, nj) : nullptr;
+        if (!(ok = mbar_wait(my_full, af, abort_flag, p.ctl))) break;
+        af ^= 1u;
+        tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            FK_TMEM_LD32(t_row + g * kTileN + c * 32, v);
-            FK_TMEM_WAIT_LD(v);
-            float cnv[32];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          FK_TMEM_LD32(t_row + c * 32, v);
+          FK_TMEM_WAIT_LD(v);
+          // chunk maximum: 3-input-max tree, depth 4
+          float l1[11];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float4 t = __ldg(cn4 + c * 8 + e);
-              cnv[4 * e] = t.x; cnv[4 * e + 1] = t.y; cnv[4 * e + 2] = t.z; cnv[4 * e + 3] = t.w;
-            }
-            int bj = -1;
+          for (int i = 0; i < 10; ++i)
+            l1[i] = fmax3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
+          l1[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+          const float l2a = fmax3(l1[0], l1[1], l1[2]), l2b = fmax3(l1[3], l1[4], l1[5]);
+          const float l2c = fmax3(l1[6], l1[7], l1[8]), l2d = fmaxf(l1[9], l1[10]);
+          const float m = fmaxf(fmax3(l2a, l2b, l2c), l2d);
+          const bool imp = m > cbest;  // strict: an earlier column keeps a tie
+          if (__any_sync(0xffffffffu, imp)) {
+            if (imp) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              const float d = fmaf(-2.f, __uint_as_float(v[t]), cnv[t]);
-              const bool lt = d < cb;
-              cb = lt ? d : cb;
-              bj = lt ? t : bj;
+              for (int t = 0; t < 32; ++t) cand[t] = v[t];
+              cbest = m;
+              cbase = col0 + c * 32;
             }
-            if (bj >= 0) bi = col0 + c * 32 + bj;
           }
-          best[g] = cb;
-          bidx[g] = bi;
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(accempty(g));
+          if (nbp) {  // the next tile's bias goes where this chunk was read
+            load_bias32(nbp + c * 32, v);
+            FK_TMEM_ST32(t_row + c * 32, v);
+          }
         }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_empty);
       }
       if (!ok) break;
-      // merge the two column halves: warpgroup wg keeps sub-tile wg
+      // lowest column of the candidate chunk holding the maximum
+      int j0 = 32, j1 = 32, j2 = 32, j3 = 32;
+#pragma unroll
+      for (int t = 28; t >= 0; t -= 4) {
+        j0 = __uint_as_float(cand[t]) == cbest ? t : j0;
+        j1 = __uint_as_float(cand[t + 1]) == cbest ? t + 1 : j1;
+        j2 = __uint_as_float(cand[t + 2]) == cbest ? t + 2 : j2;
+        j3 = __uint_as_float(cand[t + 3]) == cbest ? t + 3 : j3;
+      }
+      const int jm = min(min(j0, j1), min(j2, j3));
+      int bi = jm < 32 ? cbase + jm : 0;
+      float sb = cbest;
+      // merge the two column halves of each point: warpgroup h == 0 writes
       if (u != (int)blockIdx.x && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
-      const int give = 1 - wg;
-      xchg[give * kRowsSub + r] = make_float2(best[give], __int_as_float(bidx[give]));
+      if (h == 1) xchg[g * kRowsSub + r] = make_float2(sb, __int_as_float(bi));
       __syncwarp();
       if (lane == 0) mbar_arrive(xchg_full);
       if (!(ok = mbar_wait(xchg_full, xc, abort_flag, p.ctl))) break;
-      const float2 o = xchg[wg * kRowsSub + r];
+      if (h == 0) {
+        const float2 o = xchg[g * kRowsSub + r];
+        const int oi = __float_as_int(o.y);
+        if (o.x > sb || (o.x == sb && oi < bi)) { sb = o.x; bi = oi; }
+        const int row = r0 + g * kRowsSub + r;
+        if (row < p.N) {
+          const size_t o_ = (size_t)b * p.N + row;
+          p.labels[o_] = bi;
+          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, sb, xn));
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(xchg_empty);
-      float bb = best[wg];
-      int bi = bidx[wg];
-      const int oi = __float_as_int(o.y);
-      if (o.x < bb || (o.x == bb && oi < bi)) { bb = o.x; bi = oi; }
-      const int row = r0 + wg * kRowsSub + r;
-      if (row < p.N) {
-        const size_t o_ = (size_t)b * p.N + row;
-        p.labels[o_] = bi;
-        if (p.mindist) p.mindist[o_] = fmaxf(0.f, xn + bb);
-      }
     }
   }
 
@@ -393,7 +466,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, TcPar
   return cudaGetLastError();
 }
 
-cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *cn, int B, int N,
+cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
                              int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
                              int num_sms, cudaStream_t s) {
   if (!tc_shape_ok(dt, D) || !tc_aligned(X, C)) return cudaErrorNotSupported;
@@ -409,7 +482,7 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   p.total_units = p.upb * B;
   p.idesc = idesc_f16(dt == kBF16 ? 1 : 0, kRowsSub, kTileN);
   p.is_bf16 = dt == kBF16;
-  p.cn = cn;
+  p.bias = bias;
   p.labels = labels;
   p.mindist = mindist;
   p.ctl = ctl;

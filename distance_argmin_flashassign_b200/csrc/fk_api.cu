@@ -114,8 +114,8 @@ static int choose_path(DType dt, int D) {
   return tc_shape_ok(dt, D) ? 1 : 2;
 }
 
-// Assignment of B problems.  cn (B*Kpad norms of C) may be null, in which
-// case the tensor path computes it into scratch at `cn_ws`.
+// Assignment of B problems.  cn (the B*Kpad bias -|c|^2/2 of C) may be null,
+// in which case the tensor path computes it into scratch at `cn_ws`.
 static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
                             const float *cn, float *cn_ws, int32_t *labels, float *mindist,
                             cudaStream_t s) {
@@ -124,8 +124,8 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
   if (path == 1 && tc_aligned(X, C)) {
     const int Kpad = pad_k(K);
     if (!cn) {
-      cudaError_t e = launch_norms(dt, C, B, K, Kpad, D, cn_ws, s);
-      if (e != cudaSuccess) return cuda_fail(e, "norms kernel");
+      cudaError_t e = launch_bias(dt, C, B, K, Kpad, D, cn_ws, s);
+      if (e != cudaSuccess) return cuda_fail(e, "bias kernel");
       cn = cn_ws;
     }
     cudaError_t e = launch_assign_tc(dt, X, C, cn, B, N, D, K, Kpad, labels, mindist, ctl_of(d), d.sms, s);
@@ -201,38 +201,38 @@ fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C,
   return fk_assign_batched(X, 1, N, D, dt, C, K, labels, mindist, stream);
 }
 
-int64_t fk_norms_len(int B, int K) {
+int64_t fk_bias_len(int B, int K) {
   if (B < 1 || K < 1) return 0;
   return (int64_t)B * pad_k(K);
 }
 
-fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt, float *norms,
+fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt, float *bias,
                                fk_stream_t stream) {
   fk_status st = check_sizes(B, 0, D, K, dt);
   if (st != FK_OK) return st;
-  if (!C32 || !C_dt || !norms) return fail(FK_ERR_INVALID_ARG, "C32, C_dt and norms must not be NULL");
+  if (!C32 || !C_dt || !bias) return fail(FK_ERR_INVALID_ARG, "C32, C_dt and bias must not be NULL");
   DevState *d;
   if ((st = device_state(&d)) != FK_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const DType t = (DType)dt;
   cudaError_t e;
   if (t == kF32 && C_dt == (const void *)C32)
-    e = launch_norms(t, C32, B, K, pad_k(K), D, norms, s);
+    e = launch_bias(t, C32, B, K, pad_k(K), D, bias, s);
   else
-    e = launch_round_norms(t, C32, B, K, pad_k(K), D, C_dt, norms, s);
+    e = launch_round_bias(t, C32, B, K, pad_k(K), D, C_dt, bias, s);
   if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
   return FK_OK;
 }
 
 fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt, int K,
-                             const float *norms, int32_t *labels, float *mindist, fk_stream_t stream) {
+                             const float *bias, int32_t *labels, float *mindist, fk_stream_t stream) {
   fk_status st = check_sizes(B, N, D, K, dt);
   if (st != FK_OK) return st;
   if (N == 0) return FK_OK;
-  if (!X || !C_dt || !labels || !norms) return fail(FK_ERR_INVALID_ARG, "X, C_dt, norms and labels must not be NULL");
+  if (!X || !C_dt || !labels || !bias) return fail(FK_ERR_INVALID_ARG, "X, C_dt, bias and labels must not be NULL");
   DevState *d;
   if ((st = device_state(&d)) != FK_OK) return st;
-  return run_assign(*d, (DType)dt, X, B, (int)N, D, C_dt, K, norms, nullptr, labels, mindist, (cudaStream_t)stream);
+  return run_assign(*d, (DType)dt, X, B, (int)N, D, C_dt, K, bias, nullptr, labels, mindist, (cudaStream_t)stream);
 }
 
 fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t N, int D, fk_dtype dt,
@@ -309,7 +309,7 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   a.mode = kMean;
   for (int it = 0; it < iters; ++it) {
     if (t != kF32) {  // fp32 runs on the CUDA-core kernel, which needs no norms
-      cudaError_t e = launch_round_norms(t, C, B, K, Kpad, D, Cdt, cn, s);
+      cudaError_t e = launch_round_bias(t, C, B, K, Kpad, D, Cdt, cn, s);
       if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
     }
     st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, labels, it == iters - 1 ? mindist : nullptr, s);
@@ -405,7 +405,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
       FK_TRY(cudaMemsetAsync(acc, 0, (size_t)K * D * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
       FK_TRY(cudaMemsetAsync(cnt, 0, (size_t)K * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
       if (t != kF32)
-        FK_TRY(launch_round_norms(t, c32, 1, K, Kpad, D, cdt, cn, s), "centroid prep kernel", FK_ERR_CUDA);
+        FK_TRY(launch_round_bias(t, c32, 1, K, Kpad, D, cdt, cn, s), "centroid prep kernel", FK_ERR_CUDA);
       for (int64_t c = 0; c < nchunks; ++c) {
         const int slot = (int)(c & 1);
         const int64_t r0 = c * rows;

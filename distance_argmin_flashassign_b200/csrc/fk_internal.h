@@ -17,13 +17,13 @@ constexpr int kCentroidPad = 256;  // centroid tile of the tensor-core kernel
 inline int pad_k(int K) { return (K + kCentroidPad - 1) / kCentroidPad * kCentroidPad; }
 inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
 
-// ---- prep.cu: centroid norms (row norms of the assignment stage) ----------
-// cn[b*Kpad + j] = |C[b][j]|^2 in fp32 for j < K, +inf for K <= j < Kpad.
-cudaError_t launch_norms(DType dt, const void *C, int B, int K, int Kpad, int D, float *cn,
-                         cudaStream_t s);
-// Cdt = C32 rounded to dt (round-to-nearest-even) and cn = norms of Cdt.
-cudaError_t launch_round_norms(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
-                               float *cn, cudaStream_t s);
+// ---- prep.cu: centroid bias (row norms of the assignment stage) -----------
+// bias[b*Kpad + j] = -|C[b][j]|^2 / 2 in fp32 for j < K, -inf for K <= j < Kpad.
+cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, float *bias,
+                        cudaStream_t s);
+// Cdt = C32 rounded to dt (round-to-nearest-even) and bias of Cdt.
+cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
+                              float *bias, cudaStream_t s);
 
 // ---- assign_simt.cu: CUDA-core assignment (any dtype, any D) --------------
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
@@ -33,7 +33,7 @@ cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, in
 bool tc_shape_ok(DType dt, int D);
 bool tc_aligned(const void *X, const void *C);
 // Returns cudaErrorNotSupported if the tensor maps could not be encoded.
-cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *cn, int B, int N,
+cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
                              int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
                              int num_sms, cudaStream_t s);
 

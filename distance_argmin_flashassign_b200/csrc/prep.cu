@@ -1,25 +1,27 @@
 // prep.cu -- centroid preparation for the assignment stage.
 //
-// The expanded distance |x|^2 + |c|^2 - 2<x,c> (Flash-KMeans abstract:
-// distances are computed on the fly and fed to an online argmin) needs the
-// centroid norms |c_k|^2.  They are computed once per assignment, in fp32,
-// from the centroids exactly as the tensor cores will see them (already
-// rounded to the input type), and padded with +inf up to a multiple of the
-// 256-centroid tile so padded columns never win the argmin.
+// The tensor-core assignment ranks centroids by the score
+// s_k = <x, c_k> - |c_k|^2 / 2, which orders them exactly as the squared
+// distance |x|^2 + |c_k|^2 - 2<x, c_k> does (Flash-KMeans abstract: the
+// distance is computed on the fly and fed to an online arg-min).  The bias
+// -|c_k|^2 / 2 is computed once per assignment in fp32 from the centroids as
+// the tensor cores see them (already rounded to the input type) and padded
+// with -inf up to a multiple of the 256-centroid tile, so padded columns
+// never win.
 #include "fk_internal.h"
 
 namespace fk {
 
 template <typename T>
-__global__ void __launch_bounds__(256) norms_kernel(const T *__restrict__ C, int B, int K, int Kpad,
-                                                    int D, float *__restrict__ cn) {
+__global__ void __launch_bounds__(256) bias_kernel(const T *__restrict__ C, int B, int K, int Kpad,
+                                                    int D, float *__restrict__ bias) {
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)B * Kpad;
   for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows;
        r += (long long)gridDim.x * 8) {
     const int b = (int)(r / Kpad), j = (int)(r % Kpad);
     if (j >= K) {
-      if (lane == 0) cn[r] = __int_as_float(0x7f800000);
+      if (lane == 0) bias[r] = __int_as_float(0xff800000);
       continue;
     }
     const T *c = C + ((size_t)b * K + j) * D;
@@ -29,21 +31,21 @@ __global__ void __launch_bounds__(256) norms_kernel(const T *__restrict__ C, int
       s = fmaf(v, v, s);
     }
     s = warp_sum(s);
-    if (lane == 0) cn[r] = s;
+    if (lane == 0) bias[r] = -0.5f * s;
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) round_norms_kernel(const float *__restrict__ C32, int B, int K,
+__global__ void __launch_bounds__(256) round_bias_kernel(const float *__restrict__ C32, int B, int K,
                                                           int Kpad, int D, T *__restrict__ Cdt,
-                                                          float *__restrict__ cn) {
+                                                          float *__restrict__ bias) {
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)B * Kpad;
   for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows;
        r += (long long)gridDim.x * 8) {
     const int b = (int)(r / Kpad), j = (int)(r % Kpad);
     if (j >= K) {
-      if (lane == 0) cn[r] = __int_as_float(0x7f800000);
+      if (lane == 0) bias[r] = __int_as_float(0xff800000);
       continue;
     }
     const size_t off = ((size_t)b * K + j) * D;
@@ -55,7 +57,7 @@ __global__ void __launch_bounds__(256) round_norms_kernel(const float *__restric
       s = fmaf(v, v, s);
     }
     s = warp_sum(s);
-    if (lane == 0) cn[r] = s;
+    if (lane == 0) bias[r] = -0.5f * s;
   }
 }
 
@@ -64,32 +66,32 @@ static int grid_for_rows(long long rows) {
   return (int)(g < 4096 ? (g < 1 ? 1 : g) : 4096);
 }
 
-cudaError_t launch_norms(DType dt, const void *C, int B, int K, int Kpad, int D, float *cn,
+cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, float *bias,
                          cudaStream_t s) {
   const int g = grid_for_rows((long long)B * Kpad);
   switch (dt) {
-    case kF32: norms_kernel<float><<<g, 256, 0, s>>>((const float *)C, B, K, Kpad, D, cn); break;
-    case kF16: norms_kernel<__half><<<g, 256, 0, s>>>((const __half *)C, B, K, Kpad, D, cn); break;
+    case kF32: bias_kernel<float><<<g, 256, 0, s>>>((const float *)C, B, K, Kpad, D, bias); break;
+    case kF16: bias_kernel<__half><<<g, 256, 0, s>>>((const __half *)C, B, K, Kpad, D, bias); break;
     default:
-      norms_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)C, B, K, Kpad, D, cn);
+      bias_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)C, B, K, Kpad, D, bias);
   }
   count_launches(1);
   return cudaGetLastError();
 }
 
-cudaError_t launch_round_norms(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
-                               float *cn, cudaStream_t s) {
+cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
+                               float *bias, cudaStream_t s) {
   const int g = grid_for_rows((long long)B * Kpad);
   switch (dt) {
     case kF32:
-      round_norms_kernel<float><<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (float *)Cdt, cn);
+      round_bias_kernel<float><<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (float *)Cdt, bias);
       break;
     case kF16:
-      round_norms_kernel<__half><<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (__half *)Cdt, cn);
+      round_bias_kernel<__half><<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (__half *)Cdt, bias);
       break;
     default:
-      round_norms_kernel<__nv_bfloat16>
-          <<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (__nv_bfloat16 *)Cdt, cn);
+      round_bias_kernel<__nv_bfloat16>
+          <<<g, 256, 0, s>>>(C32, B, K, Kpad, D, (__nv_bfloat16 *)Cdt, bias);
   }
   count_launches(1);
   return cudaGetLastError();

@@ -9,16 +9,15 @@
 //      a per-digit scan over tiles, and a scatter whose within-tile ranks come
 //      from warp-level match_any -- the sorted point ids are the inverse map
 //      (cluster -> its points);
-//   2. segment offsets by a lower-bound search of every cluster id in the
-//      sorted ids;
-//   3. segmented sums: the sorted order is cut into equal chunks of R
+//   2. segmented sums: the sorted order is cut into equal chunks of R
 //      positions, one warp per chunk, so a hot cluster (Zipf skew) is spread
 //      over many warps instead of serialising on one address.  A warp gathers
 //      its rows coalesced (each row is read as one contiguous vector per
 //      lane), accumulates in fp32 registers and writes a segment that lies
 //      wholly inside its chunk straight to the output; the two boundary
-//      segments of a chunk go to partial slots;
-//   4. finalize: per cluster, partials of chunk-crossing segments are summed
+//      segments of a chunk go to partial slots.  The same warps write the
+//      segment offsets (first sorted position of every cluster id);
+//   3. finalize: per cluster, partials of chunk-crossing segments are summed
 //      in a fixed order and divided by the count; empty clusters are left
 //      untouched.  No global atomics anywhere, so results are deterministic.
 //
@@ -63,8 +62,12 @@ static SortPlan plan_sort(long long Ntot, long long Ktot) {
   return p;
 }
 
+// Positions per segment-sum warp: enough warps for about one wave of a
+// B200 (148 SMs x 12 resident warps), at least 256.  Depends on Ntot only, so
+// the summation order (and the result) does not depend on the device.
 static int chunk_rows_R(long long Ntot) {
-  long long R = (Ntot / 8192 + 31) / 32 * 32;
+  long long R = (Ntot + 1775) / 1776;
+  R = (R + 31) / 32 * 32;
   return (int)(R < 256 ? 256 : R);
 }
 
@@ -208,17 +211,20 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   }
 }
 
-// off[k] = first position of key >= k in the sorted keys, k in [0, Ktot].
-__global__ void __launch_bounds__(256) seg_offsets_kernel(const int32_t *__restrict__ skeys, int Ntot,
-                                                          int Ktot, int *__restrict__ off) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k > Ktot) return;
-  int lo = 0, hi = Ntot;
-  while (lo < hi) {
-    const int mid = lo + ((hi - lo) >> 1);
-    if (skeys[mid] < k) lo = mid + 1; else hi = mid;
-  }
-  off[k] = lo;
+// Segment offsets are written by the segment-sum warps: at every position
+// where the sorted key changes from kp to k, off[kp+1 .. k] = that position
+// (empty clusters in between share it); the warp ending at Ntot writes
+// off[k_last+1 .. Ktot] = Ntot.  Every entry is written exactly once.
+__device__ __forceinline__ void write_offsets(int *__restrict__ off, int kp, int k, int pos, int lane) {
+  for (int kk = kp + 1 + lane; kk <= k; kk += 32) off[kk] = pos;
+}
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------- segmented sums --
@@ -236,6 +242,20 @@ template <> struct Vec<float> {
       v[0] = w.x; v[1] = w.y;
     } else {
       v[0] = __ldg(p);
+    }
+  }
+  template <int N> __device__ static void load_shared(const float *p, float *v) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 4; ++i) {
+        const float4 w = reinterpret_cast<const float4 *>(p)[i];
+        v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+      }
+    } else if constexpr (N == 2) {
+      const float2 w = *reinterpret_cast<const float2 *>(p);
+      v[0] = w.x; v[1] = w.y;
+    } else {
+      v[0] = p[0];
     }
   }
 };
@@ -266,6 +286,23 @@ template <typename T, bool BF> struct Vec16 {
       v[0] = to_f32<T>(p[0]);
     }
   }
+  template <int N> __device__ static void load_shared(const T *p, float *v) {
+    auto up = [](uint32_t w, float *o) { if (BF) unpack_bf162(w, o); else unpack_half2(w, o); };
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) {
+        const uint4 w = reinterpret_cast<const uint4 *>(p)[i];
+        up(w.x, v + 8 * i); up(w.y, v + 8 * i + 2); up(w.z, v + 8 * i + 4); up(w.w, v + 8 * i + 6);
+      }
+    } else if constexpr (N == 4) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(p);
+      up(w.x, v); up(w.y, v + 2);
+    } else if constexpr (N == 2) {
+      up(*reinterpret_cast<const unsigned int *>(p), v);
+    } else {
+      v[0] = to_f32<T>(p[0]);
+    }
+  }
 };
 template <> struct Vec<__half> : Vec16<__half, false> {};
 template <> struct Vec<__nv_bfloat16> : Vec16<__nv_bfloat16, true> {};
@@ -275,9 +312,9 @@ template <> struct Vec<__nv_bfloat16> : Vec16<__nv_bfloat16, true> {};
 template <typename T, int NACC, bool CONTIG, int MODE>
 __global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, int D,
                                                      const int32_t *__restrict__ perm,
-                                                     const int32_t *__restrict__ skeys, int Ntot, int R,
-                                                     float *__restrict__ C, double *__restrict__ acc,
-                                                     float *__restrict__ parts) {
+                                                     const int32_t *__restrict__ skeys, int Ntot, int Ktot,
+                                                     int R, float *__restrict__ C, double *__restrict__ acc,
+                                                     float *__restrict__ parts, int *__restrict__ off) {
   constexpr int PF = NACC <= 4 ? 8 : (NACC <= 8 ? 4 : (NACC <= 16 ? 2 : 1));  // rows in flight
   const int lane = threadIdx.x & 31;
   const long long wq = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -286,8 +323,10 @@ __global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, in
   const int p0 = (int)p0l;
   const int p1 = (Ntot - p0) < R ? Ntot : p0 + R;
   const int kfirst = skeys[p0];
-  const bool split_start = p0 > 0 && skeys[p0 - 1] == kfirst;
+  const int kprev = p0 > 0 ? skeys[p0 - 1] : -1;
+  const bool split_start = kprev == kfirst;
   const bool split_end = p1 < Ntot && skeys[p1] == skeys[p1 - 1];
+  write_offsets(off, kprev, kfirst, p0, lane);
 
   float a[NACC];
 #pragma unroll
@@ -352,6 +391,7 @@ __global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, in
         if (t0 + u < n) {
           if (k != cur) {
             flush(cur, s, b0 + t0 + u);
+            write_offsets(off, cur, k, b0 + t0 + u, lane);
             cur = k;
             s = b0 + t0 + u;
 #pragma unroll
@@ -364,6 +404,120 @@ __global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, in
     }
   }
   flush(cur, s, p1);
+  if (p1 == Ntot) write_offsets(off, cur, Ktot, Ntot, lane);
+}
+
+// Staged variant for rows of 32*NACC elements whose byte size is a multiple
+// of 16: every warp copies the rows of its next groups of 32 sorted
+// positions into a shared-memory ring with cp.async (16 bytes per lane, no
+// registers held), so about 16 KB per warp are in flight while it sums the
+// group that has landed.
+constexpr int kSegWarps = 4, kSegStages = 2;
+template <typename T, int NACC, int MODE>
+__global__ void __launch_bounds__(kSegWarps * 32) segsum_staged_kernel(
+    const T *__restrict__ X, int D, const int32_t *__restrict__ perm, const int32_t *__restrict__ skeys, int Ntot,
+    int Ktot, int R, float *__restrict__ C, double *__restrict__ acc, float *__restrict__ parts,
+    int *__restrict__ off) {
+  constexpr int RB = 32 * NACC * (int)sizeof(T);  // bytes per row
+  constexpr int PIECES = RB / 16;
+  constexpr int SLOT = 32 * RB;
+  static_assert(RB % 16 == 0, "rows must be whole 16-byte pieces");
+  extern __shared__ __align__(16) uint8_t seg_smem[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  uint8_t *ring = seg_smem + wib * (kSegStages * SLOT);
+  const long long wq = (long long)blockIdx.x * kSegWarps + wib;
+  const long long p0l = wq * R;
+  if (p0l >= Ntot) return;
+  const int p0 = (int)p0l;
+  const int p1 = (Ntot - p0) < R ? Ntot : p0 + R;
+  const int kfirst = skeys[p0];
+  const int kprev = p0 > 0 ? skeys[p0 - 1] : -1;
+  const bool split_start = kprev == kfirst;
+  const bool split_end = p1 < Ntot && skeys[p1] == skeys[p1 - 1];
+  write_offsets(off, kprev, kfirst, p0, lane);
+  const int ngroups = (p1 - p0 + 31) / 32;
+
+  float a[NACC];
+#pragma unroll
+  for (int i = 0; i < NACC; ++i) a[i] = 0.f;
+  int cur = kfirst, s = p0;
+  auto flush = [&](int k, int sb, int se) {
+    const bool split = (sb == p0 && split_start) || (se == p1 && split_end);
+    float *dst;
+    if (!split) {
+      if (MODE == kMean) {
+        const float fc = (float)(se - sb);
+        dst = C + (size_t)k * D + lane * NACC;
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) dst[i] = a[i] / fc;
+      } else {
+        double *dd = acc + (size_t)k * D + lane * NACC;
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) dd[i] += (double)a[i];
+      }
+    } else {
+      dst = parts + ((size_t)wq * 2 + (sb == p0 ? 0 : 1)) * D + lane * NACC;
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) dst[i] = a[i];
+    }
+  };
+  // copy the rows of group g into ring slot `slot`; returns (key, row) of lane
+  auto issue = [&](int g, int slot, int &mk, int &mr) {
+    const int base = p0 + g * 32;
+    const int n = (p1 - base) < 32 ? (p1 - base) : 32;
+    mk = lane < n ? skeys[base + lane] : 0;
+    mr = lane < n ? perm[base + lane] : 0;
+    uint8_t *dst = ring + slot * SLOT;
+#pragma unroll
+    for (int it = 0; it < PIECES; ++it) {
+      const int q = it * 32 + lane;
+      const int i = q / PIECES, pc = q % PIECES;
+      const int row = __shfl_sync(0xffffffffu, mr, i);
+      if (i < n) cp_async16(dst + q * 16, reinterpret_cast<const uint8_t *>(X) + (size_t)row * RB + pc * 16);
+    }
+    cp_async_commit();
+  };
+  auto consume = [&](int g, int slot, int mk) {
+    const int base = p0 + g * 32;
+    const int n = (p1 - base) < 32 ? (p1 - base) : 32;
+    const T *src = reinterpret_cast<const T *>(ring + slot * SLOT) + lane * NACC;
+    for (int t = 0; t < n; ++t) {
+      const int k = __shfl_sync(0xffffffffu, mk, t);
+      if (k != cur) {
+        flush(cur, s, base + t);
+        write_offsets(off, cur, k, base + t, lane);
+        cur = k;
+        s = base + t;
+#pragma unroll
+        for (int i = 0; i < NACC; ++i) a[i] = 0.f;
+      }
+      float v[NACC];
+      Vec<T>::template load_shared<NACC>(src + t * (32 * NACC), v);
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) a[i] += v[i];
+    }
+  };
+
+  int k0 = 0, r0 = 0, k1 = 0, r1 = 0;
+  issue(0, 0, k0, r0);
+  if (ngroups > 1) issue(1, 1, k1, r1);
+  for (int g = 0; g < ngroups; g += 2) {
+    // slot 0 holds group g
+    if (g + 1 < ngroups) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncwarp();
+    consume(g, 0, k0);
+    __syncwarp();
+    if (g + 2 < ngroups) issue(g + 2, 0, k0, r0);
+    if (g + 1 >= ngroups) break;
+    // slot 1 holds group g + 1
+    if (g + 2 < ngroups) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncwarp();
+    consume(g + 1, 1, k1);
+    __syncwarp();
+    if (g + 3 < ngroups) issue(g + 3, 1, k1, r1);
+  }
+  flush(cur, s, p1);
+  if (p1 == Ntot) write_offsets(off, cur, Ktot, Ntot, lane);
 }
 
 // One block per cluster (grid-stride): counts, then the fixed-order sum of
@@ -464,18 +618,42 @@ size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D) {
   return carve(nullptr, Ntot, Ktot, D).bytes;
 }
 
-template <typename T, int MODE>
-static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_t *skeys, int Ntot, int R,
-                          float *parts, cudaStream_t s) {
+template <typename T, int MODE, int NACC>
+static void launch_staged(const UpdateArgs &a, const int32_t *perm, const int32_t *skeys, int Ntot, int Ktot,
+                          int R, float *parts, int *off, cudaStream_t s) {
+  constexpr int smem = kSegWarps * kSegStages * 32 * 32 * NACC * (int)sizeof(T);
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaFuncSetAttribute(segsum_staged_kernel<T, NACC, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    configured[dev] = true;
+  }
   const long long nchunks = ((long long)Ntot + R - 1) / R;
-  const int grid = (int)((nchunks + 7) / 8);
+  const int grid = (int)((nchunks + kSegWarps - 1) / kSegWarps);
+  segsum_staged_kernel<T, NACC, MODE><<<grid, kSegWarps * 32, smem, s>>>((const T *)a.X, a.D, perm, skeys, Ntot,
+                                                                        Ktot, R, a.C, a.acc, parts, off);
+}
+
+template <typename T, int MODE>
+static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_t *skeys, int Ntot, int Ktot,
+                          int R, float *parts, int *off, cudaStream_t s) {
   const T *X = (const T *)a.X;
   const int D = a.D;
-  const size_t es = sizeof(T);
-  const bool contig_ok = D % 32 == 0 && ((uintptr_t)a.X % 16 == 0);
-  const int nacc_c = D / 32;
+  const bool aligned = ((uintptr_t)a.X % 16 == 0);
+  const int nacc_c = D % 32 == 0 ? D / 32 : 0;
+  const int rb = nacc_c * (int)sizeof(T) * 32;
+  if (aligned && rb % 16 == 0 && rb > 0 && rb <= 512) {
+    if (nacc_c == 1) return launch_staged<T, MODE, 1>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
+    if (nacc_c == 2) return launch_staged<T, MODE, 2>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
+    if (nacc_c == 4) return launch_staged<T, MODE, 4>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
+    if (nacc_c == 8 && sizeof(T) == 2) return launch_staged<T, MODE, 8>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
+  }
+  const long long nchunks = ((long long)Ntot + R - 1) / R;
+  const int grid = (int)((nchunks + 7) / 8);
+  const bool contig_ok = D % 32 == 0 && aligned;
 #define FK_SEG(NA, CG) \
-  segsum_kernel<T, NA, CG, MODE><<<grid, 256, 0, s>>>(X, D, perm, skeys, Ntot, R, a.C, a.acc, parts)
+  segsum_kernel<T, NA, CG, MODE><<<grid, 256, 0, s>>>(X, D, perm, skeys, Ntot, Ktot, R, a.C, a.acc, parts, off)
   if (contig_ok && nacc_c == 1) FK_SEG(1, true);
   else if (contig_ok && nacc_c == 2) FK_SEG(2, true);
   else if (contig_ok && nacc_c == 4) FK_SEG(4, true);
@@ -490,7 +668,6 @@ static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_
     else FK_SEG(32, false);
   }
 #undef FK_SEG
-  (void)es;
 }
 
 cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl ctl, int num_sms,
@@ -530,20 +707,20 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
     vout = (vout == w.vA) ? w.vB : w.vA;
   }
   const int32_t *skeys = kin, *perm = vin;
-  seg_offsets_kernel<<<(int)((Ktot + 1 + 255) / 256), 256, 0, s>>>(skeys, N, (int)Ktot, w.off);
   const int R = chunk_rows_R(Ntot);
+  const int KT = (int)Ktot;
   switch (a.dt) {
     case kF32:
-      a.mode == kMean ? launch_segsum<float, kMean>(a, perm, skeys, N, R, w.parts, s)
-                      : launch_segsum<float, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+      a.mode == kMean ? launch_segsum<float, kMean>(a, perm, skeys, N, KT, R, w.parts, w.off, s)
+                      : launch_segsum<float, kAccumulate>(a, perm, skeys, N, KT, R, w.parts, w.off, s);
       break;
     case kF16:
-      a.mode == kMean ? launch_segsum<__half, kMean>(a, perm, skeys, N, R, w.parts, s)
-                      : launch_segsum<__half, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+      a.mode == kMean ? launch_segsum<__half, kMean>(a, perm, skeys, N, KT, R, w.parts, w.off, s)
+                      : launch_segsum<__half, kAccumulate>(a, perm, skeys, N, KT, R, w.parts, w.off, s);
       break;
     default:
-      a.mode == kMean ? launch_segsum<__nv_bfloat16, kMean>(a, perm, skeys, N, R, w.parts, s)
-                      : launch_segsum<__nv_bfloat16, kAccumulate>(a, perm, skeys, N, R, w.parts, s);
+      a.mode == kMean ? launch_segsum<__nv_bfloat16, kMean>(a, perm, skeys, N, KT, R, w.parts, w.off, s)
+                      : launch_segsum<__nv_bfloat16, kAccumulate>(a, perm, skeys, N, KT, R, w.parts, w.off, s);
   }
   const int fgrid = (int)(Ktot < (long long)num_sms * 4 ? Ktot : (long long)num_sms * 4);
   if (a.mode == kMean)
@@ -552,7 +729,7 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
   else
     seg_finalize_kernel<kAccumulate><<<fgrid, 512, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr,
                                                            nullptr, a.acc, a.cnt);
-  nl += 3;
+  nl += 2;
   count_launches(nl);
   return cudaGetLastError();
 }

@@ -27,8 +27,8 @@
  *              a CUDA-core kernel (fp32 always does).
  *   Distances  label[i] = argmin_k |x_i - c_k|^2 with ties to the LOWEST k
  *              (the pages are silent on ties).  mindist[i] = that squared
- *              distance, clamped at 0.  The tensor path evaluates
- *              |c|^2 - 2<x,c> (+|x|^2 for mindist) in fp32.
+ *              distance, clamped at 0.  The tensor path ranks by
+ *              <x,c> - |c|^2/2 in fp32 (mindist = |x|^2 - 2 * best score).
  *   Update     C_k = mean of the points with label k, in fp32; a cluster
  *              that receives no point keeps its previous centroid and gets
  *              count 0 (the pages are silent on empty clusters).
@@ -112,23 +112,25 @@ FK_API fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dt
 /* ------------------------------------------------------------------------
  * Two-phase assignment for callers that iterate (Lloyd loops, benchmarks).
  *
- * fk_norms_len -- number of floats of the norm buffer for B problems of K
+ * fk_bias_len -- number of floats of the bias buffer for B problems of K
  *   centroids (K rounded up to the 256-centroid tile, per problem).
  * fk_prepare_centroids -- the preparation step of the assignment stage:
  *   C_dt = C32 rounded to dt (round-to-nearest-even; a plain copy for
- *   FK_F32, skipped when C_dt == C32) and norms = |C_dt[k]|^2 in fp32, with
- *   +inf in the padding so padded columns never win.  One kernel.
- *   C32 device B x K x D fp32; C_dt device B x K x D of dt; norms device
- *   fk_norms_len(B, K) floats.
+ *   FK_F32, skipped when C_dt == C32) and bias = -|C_dt[k]|^2 / 2 in fp32,
+ *   with -inf in the padding so padded columns never win.  The tensor-core
+ *   kernel ranks centroids by <x, c> + bias, which orders them exactly as the
+ *   squared distance does.  One kernel.
+ *   C32 device B x K x D fp32; C_dt device B x K x D of dt; bias device
+ *   fk_bias_len(B, K) floats.
  * fk_assign_prepared -- fk_assign_batched against prepared centroids and
- *   norms; launches exactly one kernel (the CUDA-core kernel, which computes
- *   direct differences, does not read the norms).
+ *   bias; launches exactly one kernel (the CUDA-core kernel, which computes
+ *   direct differences, does not read the bias).
  * ------------------------------------------------------------------------ */
-FK_API int64_t fk_norms_len(int B, int K);
+FK_API int64_t fk_bias_len(int B, int K);
 FK_API fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt,
-                                      float *norms, fk_stream_t stream);
+                                      float *bias, fk_stream_t stream);
 FK_API fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt,
-                                    int K, const float *norms, int32_t *labels, float *mindist,
+                                    int K, const float *bias, int32_t *labels, float *mindist,
                                     fk_stream_t stream);
 
 /* ------------------------------------------------------------------------

@@ -10,7 +10,7 @@ import torch
 import distance_argmin_flashassign_b200 as fk
 import oracle
 import workloads
-from tests.parity import TORCH_DT, check_centroids, check_labels, f64, rel_l2
+from tests.parity import TORCH_DT, centroid_slack, check_centroids, check_labels, f64, rel_l2
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -155,23 +155,47 @@ def test_update_reports_bad_label():
     fk.fk_sync()  # the status word was cleared
 
 
-@pytest.mark.parametrize("cfg,N,K,iters,nc", [
+LLOYD_CASES = [
     ("tiny_f32", 32768, 128, 5, 128),          # the tiny workload at full size
     ("embed_f16", 16384, 256, 3, 256),
     ("zipf_bf16", 16384, 1024, 2, 1024),
-])
-def test_lloyd_matches_oracle(cfg, N, K, iters, nc):
+]
+
+
+@pytest.mark.parametrize("cfg,N,K,iters,nc", LLOYD_CASES)
+def test_lloyd_step_by_step(cfg, N, K, iters, nc):
+    """One GPU Lloyd step at a time, each started from the oracle's centroids
+    of that step (inputs flow from the oracle to the GPU only)."""
+    s = workloads.spec(cfg, N=N, K=K, n_centers=nc)
+    w = workloads.make(s, seed=0)
+    X64 = f64(w.X)
+    Xd = w.X.to(DEV)
+    C = f64(w.C0)
+    for t in range(iters):
+        C_next, lab, mind, _, counts = oracle.lloyd_step(X64, C, s.dtype)
+        Cg = torch.from_numpy(C.astype(np.float32)).to(DEV)
+        Cg, labels, gmind, gcounts = fk.fk_lloyd(Xd, Cg, 1, want_mindist=True)
+        check_labels(X64, oracle.round_to(s.dtype, C), labels, s.dtype, gpu_mindist=gmind)
+        slack = centroid_slack(X64, lab, labels.cpu().numpy(), C_next, counts)
+        check_centroids(Cg, C_next, tol=1e-4 + slack)
+        assert int(gcounts.sum()) == N
+        assert torch.equal(gcounts.cpu().long(), torch.bincount(labels.cpu().long(), minlength=K))
+        C = C_next
+
+
+@pytest.mark.parametrize("cfg,N,K,iters,nc", LLOYD_CASES[:2])
+def test_lloyd_trajectory_matches_oracle(cfg, N, K, iters, nc):
+    """Whole fk_lloyd runs against the oracle's own trajectory (workloads whose
+    clusters are well separated, so the two trajectories cannot part)."""
     s = workloads.spec(cfg, N=N, K=K, n_centers=nc)
     w = workloads.make(s, seed=0)
     C = w.C0.clone().to(DEV)
     C, labels, mind, counts = fk.fk_lloyd(w.X.to(DEV), C, iters, want_mindist=True)
     out = oracle.lloyd(f64(w.X), f64(w.C0), iters, s.dtype)
     check_centroids(C, out["C"])
-    # the last assignment was made against C_{iters-1}: rebuild it from the oracle trajectory
     Cprev = oracle.lloyd(f64(w.X), f64(w.C0), iters - 1, s.dtype)["C"] if iters > 1 else f64(w.C0)
     check_labels(f64(w.X), oracle.round_to(s.dtype, Cprev), labels, s.dtype, gpu_mindist=mind)
     assert int(counts.sum()) == N
-    assert torch.equal(counts.cpu().long(), torch.bincount(labels.cpu().long(), minlength=K))
 
 
 def test_lloyd_batched_matches_oracle():
