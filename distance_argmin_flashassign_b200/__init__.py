@@ -50,6 +50,7 @@ def _load():
         "fk_assign_batched": [V, I, I64, I, I, V, I, V, V, V],
         "fk_update": [V, V, I64, I, I, I, V, V, V],
         "fk_update_batched": [V, V, I, I64, I, I, I, V, V, V],
+        "fk_update_noalloc": [V, V, I64, I, I, I, V, V, V],
         "fk_lloyd": [V, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_batched": [V, I, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_ooc": [V, I64, I, I, V, I, V, V, I, I64, V],
@@ -82,7 +83,7 @@ def _load():
 lib = _load()
 
 # names declared in include/fk.h (the C ABI this binding mirrors)
-ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_lloyd",
+ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_version")
@@ -187,6 +188,25 @@ def fk_update(X, labels, C, counts=None, stream=None):
                                      _stream(stream)))
     else:
         _check(lib.fk_update(_ptr(X), _ptr(labels), N, D, _dtype(X), K, _ptr(C), _ptr(counts), _stream(stream)))
+    return C, counts
+
+
+def fk_update_noalloc(X, labels, C, counts=None, stream=None):
+    """fk_update without any device allocation by the library: its scratch is a
+    fixed 32 MiB array inside libfk (about 1.5 M points at D = 128).  For
+    callers that cannot let a library allocate (stream capture, a framework
+    that owns all device memory, allocation-free loops).  Calls sharing that
+    array must not overlap on the GPU."""
+    B, N, D, bat = _dims(X)
+    if bat:
+        raise ValueError("fk_update_noalloc takes one problem (N x D)")
+    K = C.shape[-2]
+    _need(labels, "labels", torch.int32, (N,), X.device)
+    _need(C, "C", torch.float32, (K, D), X.device)
+    if counts is not None:
+        _need(counts, "counts", torch.int32, (K,), X.device)
+    _check(lib.fk_update_noalloc(_ptr(X), _ptr(labels), N, D, _dtype(X), K, _ptr(C), _ptr(counts),
+                                 _stream(stream)))
     return C, counts
 
 

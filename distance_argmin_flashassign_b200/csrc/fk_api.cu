@@ -28,6 +28,10 @@ static fk_status fail(fk_status s, const std::string &msg) {
   return s;
 }
 
+// Record a non-OK status as the calling thread's last error (used by entry
+// points defined in other files).
+int record_error(int status, const char *msg) { return fail(status, msg); }
+
 static fk_status cuda_fail(cudaError_t e, const char *where) {
   const fk_status s = e == cudaErrorMemoryAllocation ? FK_ERR_OOM : FK_ERR_CUDA;
   return fail(s, std::string(where) + ": " + cudaGetErrorString(e));

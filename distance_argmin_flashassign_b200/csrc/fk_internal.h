@@ -12,6 +12,8 @@
 namespace fk {
 
 void count_launches(int n);
+// Set the calling thread's last error (fk_get_last_error / fk_last_error_message).
+int record_error(int status, const char *msg);
 
 constexpr int kCentroidPad = 256;  // centroid tile of the tensor-core kernel
 inline int pad_k(int K) { return (K + kCentroidPad - 1) / kCentroidPad * kCentroidPad; }

@@ -159,6 +159,36 @@ FK_API fk_status fk_update_batched(const void *X, const int32_t *labels, int B, 
                             fk_dtype dt, int K, float *C, int32_t *counts, fk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fk_update_noalloc -- fk_update for callers that must not allocate.
+ *   The paper has no counterpart: this entry point exists for users whose
+ *   code cannot tolerate a library allocating device memory (work recorded
+ *   under CUDA stream capture, frameworks that own all device memory through
+ *   their own pool, loops that cannot afford an allocation or the implicit
+ *   synchronisation of freeing).  It computes exactly what fk_update computes
+ *   for one problem, with the same kernels and the same arguments, but takes
+ *   its scratch from a 32 MiB array compiled into the library instead of the
+ *   allocation cache; it calls no cudaMalloc, cudaFree or other allocating
+ *   routine.
+ *   Limits: the scratch needed (about 16 bytes per point plus small tables)
+ *   must fit the 32 MiB array -- about 1.5 million points at D = 128; larger
+ *   requests return FK_ERR_UNSUPPORTED with the needed size in
+ *   fk_last_error_message().
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (no allocation); make that first call before any stream capture.  The
+ *   array exists on every device where the library's code was loaded and is
+ *   held until the process exits.
+ *   Sharing: all calls in the process share the one array and it keeps the
+ *   last call's contents; calls that can overlap on the GPU (different
+ *   streams, or different host threads on one device) race and corrupt each
+ *   other -- order them on one stream.
+ *   Errors: argument errors as fk_update.  Labels outside [0, K) are counted
+ *   in cluster 0 like fk_update, but this variant does not report them
+ *   through fk_sync().  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_update_noalloc(const void *X, const int32_t *labels, int64_t N, int D, fk_dtype dt, int K,
+                                   float *C, int32_t *counts, fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * fk_lloyd -- `iters` Lloyd iterations, device resident.
  *   Iteration t assigns X against C_t rounded (round-to-nearest-even) to the
  *   input type (fp16/bf16; fp32 uses C_t as is), then sets C_{t+1} = the
