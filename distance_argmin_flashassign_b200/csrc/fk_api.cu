@@ -40,6 +40,9 @@ static fk_status cuda_fail(cudaError_t e, const char *where) {
 struct Scratch {
   void *ptr = nullptr;
   size_t bytes = 0;
+  // out-of-core driver: side copy stream and ring events, created on first use
+  cudaStream_t copy = nullptr;
+  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
 };
 
 struct DevState {
@@ -92,6 +95,22 @@ static fk_status scratch(DevState &d, cudaStream_t s, size_t need, void **out) {
     w.bytes = want;
   }
   *out = w.ptr;
+  return FK_OK;
+}
+
+// Copy stream and events of the out-of-core driver for (device, stream).
+static fk_status ooc_streams(DevState &d, cudaStream_t s, Scratch **out) {
+  std::lock_guard<std::mutex> g(d.mu);
+  Scratch &w = d.scratch[s];
+  if (!w.copy) {
+    cudaError_t e = cudaStreamCreateWithFlags(&w.copy, cudaStreamNonBlocking);
+    for (int i = 0; e == cudaSuccess && i < 2; ++i) {
+      e = cudaEventCreateWithFlags(&w.ready[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&w.freed[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "out-of-core stream/event creation");
+  }
+  *out = &w;
   return FK_OK;
 }
 
@@ -351,7 +370,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   const size_t es = dtype_size(t);
   const int Kpad = pad_k(K);
 
-  // device buffers owned by this call
+  // device buffers, carved from the scratch cache of (device, stream)
   const size_t b_ring = al256((size_t)rows * D * es), b_lab = al256((size_t)rows * 4);
   const size_t b_c32 = al256((size_t)K * D * 4), b_cdt = t == kF32 ? 0 : al256((size_t)K * D * es);
   const size_t b_cn = al256((size_t)Kpad * 4), b_acc = al256((size_t)K * D * 8);
@@ -359,11 +378,15 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   const size_t b_upd = al256(update_workspace_bytes(rows, K, D));
   const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd;
 
-  cudaStream_t cs = nullptr;
-  cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  Scratch *sc = nullptr;
   char *mem = nullptr;
   fk_status rc = FK_OK;
   cudaError_t e;
+  if ((rc = ooc_streams(*d, s, &sc)) != FK_OK) return rc;
+  if ((rc = scratch(*d, s, total, (void **)&mem)) != FK_OK) return rc;
+  {
+    cudaStream_t cs = sc->copy;
+    cudaEvent_t *ready = sc->ready, *freed = sc->freed;
 #define FK_TRY(call, what, code)        \
   do {                                  \
     e = (call);                         \
@@ -372,13 +395,6 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
       goto done;                        \
     }                                   \
   } while (0)
-  {
-    FK_TRY(cudaMallocAsync((void **)&mem, total, s), "cudaMallocAsync(out-of-core buffers)", FK_ERR_OOM);
-    FK_TRY(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking), "cudaStreamCreate", FK_ERR_CUDA);
-    for (int i = 0; i < 2; ++i) {
-      FK_TRY(cudaEventCreateWithFlags(&ready[i], cudaEventDisableTiming), "cudaEventCreate", FK_ERR_CUDA);
-      FK_TRY(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming), "cudaEventCreate", FK_ERR_CUDA);
-    }
     char *p = mem;
     char *ring[2] = {p, p + b_ring};
     p += 2 * b_ring;
@@ -392,7 +408,8 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
     int32_t *cnts = (int32_t *)p; p += b_counts;
     void *upd = (void *)p;
 
-    // Make the allocation visible to the copy stream before it is used there.
+    // Order the copy stream after everything already queued on `s` (the
+    // scratch may just have been allocated there, or read by an earlier call).
     FK_TRY(cudaEventRecord(freed[0], s), "cudaEventRecord", FK_ERR_CUDA);
     FK_TRY(cudaEventRecord(freed[1], s), "cudaEventRecord", FK_ERR_CUDA);
     FK_TRY(cudaMemcpyAsync(c32, C_host, (size_t)K * D * 4, cudaMemcpyHostToDevice, s), "copy of C to the device",
@@ -444,17 +461,9 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   }
 done:
 #undef FK_TRY
-  if (cs) {
-    cudaStreamSynchronize(cs);
-    cudaStreamDestroy(cs);
-  }
-  if (mem) {
-    cudaFreeAsync(mem, s);
+  if (rc != FK_OK) {  // leave nothing of this call running on the side stream
+    cudaStreamSynchronize(sc->copy);
     cudaStreamSynchronize(s);
-  }
-  for (int i = 0; i < 2; ++i) {
-    if (ready[i]) cudaEventDestroy(ready[i]);
-    if (freed[i]) cudaEventDestroy(freed[i]);
   }
   return rc;
 }
@@ -519,8 +528,16 @@ fk_status fk_release_workspace(void) {
   for (auto &kv : d->scratch) {
     if (kv.second.ptr) cudaFreeAsync(kv.second.ptr, kv.first);
   }
-  d->scratch.clear();
   cudaError_t e = cudaDeviceSynchronize();
+  for (auto &kv : d->scratch) {  // the out-of-core side streams are idle now
+    Scratch &w = kv.second;
+    if (w.copy) cudaStreamDestroy(w.copy);
+    for (int i = 0; i < 2; ++i) {
+      if (w.ready[i]) cudaEventDestroy(w.ready[i]);
+      if (w.freed[i]) cudaEventDestroy(w.freed[i]);
+    }
+  }
+  d->scratch.clear();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   return FK_OK;
 }

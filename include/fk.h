@@ -222,9 +222,10 @@ FK_API fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dty
  *   C_host       host, K x D fp32, in/out
  *   labels_host  host, N int32 (out, last iteration) or NULL
  *   counts_host  host, K int32 (out) or NULL
- *   chunk_rows   rows per chunk, >= 1 (clamped to N); the library allocates
- *                2 chunk buffers plus per-chunk scratch and frees them before
- *                returning.
+ *   chunk_rows   rows per chunk, >= 1 (clamped to N); the 2 chunk buffers and
+ *                the per-chunk scratch come from the library's scratch cache
+ *                for (device, stream), kept for later calls (fk_release_workspace
+ *                frees it), together with a side copy stream and its events.
  *   Synchronous: returns when C_host (and labels/counts) are written.
  * ------------------------------------------------------------------------ */
 FK_API fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float *C_host, int K,

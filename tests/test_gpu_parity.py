@@ -230,6 +230,29 @@ def test_ooc_matches_in_core(dtype):
     assert int(cnt_h.sum()) == N
 
 
+def test_ooc_repeated_calls_and_workspace_release():
+    # The out-of-core driver keeps its buffers, side stream and events in the
+    # scratch cache: repeated calls reuse them, and a call after
+    # fk_release_workspace builds them again.  Every call gives the same result.
+    N, D, K = 20000, 64, 100
+    s = workloads.spec("ooc_f16", N=N, D=D, K=K, n_centers=K, dtype="f16")
+    w = workloads.make(s, seed=9)
+    Xh = w.X.pin_memory()
+    results = []
+    for release in (False, False, True, False):
+        if release:
+            fk.fk_release_workspace()
+        Ch = w.C0.clone()
+        lab_h = torch.empty(N, dtype=torch.int32).pin_memory()
+        fk.fk_lloyd_ooc(Xh, Ch, 1, 7000, lab_h)
+        results.append((Ch, lab_h.clone()))
+    for Ch, lab in results[1:]:
+        assert torch.equal(Ch, results[0][0])
+        assert torch.equal(lab, results[0][1])
+    out = oracle.lloyd(f64(w.X), f64(w.C0), 1, "f16")
+    check_centroids(results[0][0], out["C"])
+
+
 def test_edge_cases():
     # K = 1: every label 0, centroid = mean
     X = torch.randn(777, 16, device=DEV, dtype=torch.float16)
