@@ -8,37 +8,42 @@
 //   * clusters of two CTAs (one per SM) loop over "units" of 256 points; the
 //     leader CTA owns rows [0,128) of a unit, the peer rows [128,256);
 //   * in each CTA a TMA warp loads its 128 rows of X once per unit (kept
-//     resident while every centroid tile streams past) and its half of every
-//     256-centroid tile (128 centroids) through a ring of 16 KB stages
-//     (128-byte swizzle, one 64-element k-block per stage);
-//   * one thread of the leader issues tcgen05.mma with cta_group::2
-//     (M = 256 across the pair, N = 256, K = 16, fp32 accumulate); each CTA's
-//     TMEM receives its 128 rows x 256 columns.  Two such accumulators (all
-//     512 TMEM columns) alternate over the tiles, and a tile ends with one
-//     tcgen05.commit that reaches both CTAs.  There is no other commit: the
-//     epilogue frees a tile's centroid stages once it has seen the tile
+//     resident while every centroid tile streams past) and, per 256-centroid
+//     tile, its half (128 centroids) into a ring of tile slots: the k-blocks
+//     of the centroids (128-byte swizzle, 64 elements each) and their bias
+//     terms (32-byte rows: three tf32-exact terms of -|c|^2/2, then zeros);
+//   * one thread of the leader issues the tile's MMAs with cta_group::2
+//     (M = 256 across the pair, N = 256, fp32 accumulate; each CTA's TMEM
+//     receives its 128 rows x 256 columns).  The first, of kind tf32 and
+//     K = 8, multiplies a constant block of ones by the bias terms and so
+//     overwrites the accumulator with -|c|^2/2 (exactly: the terms and their
+//     partial sums are fp32-exact); the kind::f16 MMAs (K = 16) then add
+//     <x,c>.  The accumulator ends holding the score s = <x,c> - |c|^2/2,
+//     whose arg-max is the arg-min of |x - c|^2, and the epilogue has no
+//     per-column arithmetic left but the arg-max.  (Giving every thread the
+//     bias instead would move 128 bytes per thread per 32 columns through
+//     L1, as much as L1 returns to the registers in a whole tile.)  Two
+//     accumulators (all 512 TMEM columns) alternate over the tiles, and a
+//     tile ends with one tcgen05.commit that reaches both CTAs.  There is no
+//     other commit: the epilogue frees a tile slot once it has seen the tile
 //     complete, and a unit's X buffer once it is done with the unit;
-//   * every accumulator already holds the bias -|c|^2/2 of its columns when
-//     the MMA starts, so it ends holding the score s = <x,c> - |c|^2/2, whose
-//     arg-max is the arg-min of |x - c|^2;
 //   * eight epilogue warps per CTA: warp (h, q) owns TMEM lanes [32q, 32q+32)
 //     (one point per thread) and columns [128h, 128h+128) of every tile, read
-//     as four 32-column chunks with the next chunk's tcgen05.ld in flight
-//     while the current one is reduced.  A 3-input-max tree gives the chunk
-//     maximum; when it beats the point's running maximum (strict ">", so an
-//     earlier column keeps a tie) the lane copies the chunk into a
-//     register-resident candidate.  Right after reading a chunk the thread
-//     writes the bias of the tile that uses this accumulator next into the
-//     same columns (tcgen05.st).  The lowest column of the candidate holding
-//     the maximum is found once per unit, and the two column halves of a
-//     point are merged at the end of the unit (score, then lower index),
+//     as two pairs of 32-column chunks.  A 3-input-max tree gives the chunk
+//     maximum; when it beats the point's running maximum (strict
+//     ">", so an earlier column keeps a tie) the lane copies the chunk into a
+//     register-resident candidate.  The lowest column of the candidate
+//     holding the maximum is found once per unit, and the two column halves
+//     of a point are merged at the end of the unit (score, then lower index),
 //     together with |x|^2 for the returned squared distance;
-//   * an accumulator goes back to the MMA thread when all 16 epilogue warps
-//     of the pair have drained and re-armed it.  The peer's warps signal the
-//     leader's barrier with a relaxed cluster-scope arrive, after
-//     tcgen05.wait::ld / wait::st and tcgen05.fence::before_thread_sync: a
-//     release at cluster scope would cost more than a third of a tile, and
-//     those TMEM accesses are already complete when the arrive is issued.
+//   * nothing is written back to TMEM, so an accumulator goes back to the MMA
+//     thread as soon as all 16 epilogue warps of the pair have LOADED their
+//     last chunk pair: the reduction of that pair overlaps the next tile's
+//     MMAs.  The peer's warps signal the leader's barrier with a relaxed
+//     cluster-scope arrive, after tcgen05.wait::ld and
+//     tcgen05.fence::before_thread_sync: a release at cluster scope would cost
+//     more than a third of a tile, and those TMEM reads are already complete
+//     when the arrive is issued.
 //
 // Only labels (and optionally |x|^2 - 2 max s) leave the chip.  X, C and the
 // bias are read; nothing else is written.
@@ -61,6 +66,9 @@ constexpr int kHalfN = kTileN / 2;          // centroids per CTA per tile
 constexpr int kBlkK = 64;                   // elements per k-block (128 bytes)
 constexpr int kXBytes = kRows * 128;        // one X k-block, 16 KB
 constexpr int kStageBytes = kHalfN * 128;   // one centroid half k-block, 16 KB
+constexpr int kBiasRow = kBiasTerms * 4;    // bias terms of one centroid, 32 bytes
+constexpr int kBiasBytes = kHalfN * kBiasRow;  // bias terms of a half tile, 4 KB
+constexpr int kOnesBytes = 256;             // the tf32 A operand of the bias step
 constexpr int kAcc = 2;                     // accumulators
 constexpr int kEpiWarps = 8;                // column half x lane quarter
 constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
@@ -71,16 +79,17 @@ static_assert(kAcc * kTileN <= (int)kTmemCols, "accumulators exceed TMEM");
 static_assert(kTileN == kCentroidPad, "the bias is padded to whole tiles");
 
 template <int KB> struct TcCfg {
-  static constexpr int XBUF = 2;                 // X double buffer (next unit prefetch)
-  static constexpr int NST = KB == 1 ? 11 : 9;   // centroid stages (16 KB)
+  static constexpr int XBUF = 2;                   // X double buffer (next unit prefetch)
+  static constexpr int SLOT = KB * kStageBytes + kBiasBytes;  // one tile's centroids and bias terms
+  static constexpr int NSLOT = KB == 1 ? 9 : 4;    // tile slots in the ring
   static constexpr int X_BYTES = XBUF * KB * kXBytes;
-  static constexpr int C_BYTES = NST * kStageBytes;
-  static constexpr int XCHG_BYTES = kRows * 16;  // one float4 per row
-  // full/empty per stage, xfull/xempty per X buffer, accfull/accempty per
+  static constexpr int C_BYTES = NSLOT * SLOT;
+  static constexpr int XCHG_BYTES = kRows * 16;    // one float4 per row
+  // full/empty per slot, xfull/xempty per X buffer, accfull/accempty per
   // accumulator, xchg full/empty, drain
-  static constexpr int NBAR = 2 * NST + 2 * XBUF + 2 * kAcc + 2 + 1;
-  static constexpr int USED = X_BYTES + C_BYTES + XCHG_BYTES + NBAR * 8 + 16;
-  static_assert(NST >= KB, "a whole centroid tile must fit in the stage ring");
+  static constexpr int NBAR = 2 * NSLOT + 2 * XBUF + 2 * kAcc + 2 + 1;
+  static constexpr int USED = X_BYTES + C_BYTES + XCHG_BYTES + kOnesBytes + NBAR * 8 + 16;
+  static_assert(SLOT % 1024 == 0, "slots keep the 1 KB alignment of the 128-byte swizzle");
   static_assert(USED + 1024 <= 232448, "shared memory (227 KB per CTA on sm_100) exceeded");
 };
 
@@ -90,37 +99,60 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Maximum of 32 scores: a 3-input-max tree of depth 4.
+// Maximum of 32 scores: four interleaved chains of 3-input max over eight
+// values each (few live temporaries), then their maximum.
 __device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
-  float l1[11];
+  float m[4];
 #pragma unroll
-  for (int i = 0; i < 10; ++i)
-    l1[i] = fmax3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
-  l1[10] = fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31]));
-  const float l2a = fmax3(l1[0], l1[1], l1[2]), l2b = fmax3(l1[3], l1[4], l1[5]);
-  const float l2c = fmax3(l1[6], l1[7], l1[8]), l2d = fmaxf(l1[9], l1[10]);
-  return fmaxf(fmax3(l2a, l2b, l2c), l2d);
+  for (int c = 0; c < 4; ++c)
+    m[c] = fmax3(__uint_as_float(v[8 * c]), __uint_as_float(v[8 * c + 1]), __uint_as_float(v[8 * c + 2]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) m[c] = fmax3(m[c], __uint_as_float(v[8 * c + 3]), __uint_as_float(v[8 * c + 4]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) m[c] = fmax3(m[c], __uint_as_float(v[8 * c + 5]), __uint_as_float(v[8 * c + 6]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) m[c] = fmaxf(m[c], __uint_as_float(v[8 * c + 7]));
+  return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
 }
 
-// 32 consecutive bias values (uniform address across the warp, L1 cached).
-__device__ __forceinline__ void load_bias32(const float *p, uint32_t (&w)[32]) {
-  const float4 *p4 = reinterpret_cast<const float4 *>(p);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float4 t = __ldg(p4 + e);
-    w[4 * e] = __float_as_uint(t.x);
-    w[4 * e + 1] = __float_as_uint(t.y);
-    w[4 * e + 2] = __float_as_uint(t.z);
-    w[4 * e + 3] = __float_as_uint(t.w);
-  }
+// Pair MMA of kind tf32 (K = 8 per instruction), same operand split as the
+// kind::f16 form.
+__device__ __forceinline__ void tc_mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor of kind::tf32: fp32 accumulator, A and B tf32, both
+// K-major, shape M x N.
+constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of the bias terms as TMA writes them: K-major rows
+// of 32 bytes with the 32-byte swizzle (layout type 6), 8-row groups 256 B
+// apart.  The base must be 256-byte aligned.
+__device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(256 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)6 << 61);
+}
+
+// Shared-memory descriptor of the block of ones, without swizzle: the two
+// 16-byte column groups of a row are core matrices 128 B apart (leading byte
+// offset) and every 8-row group reads the same 8 rows (stride byte offset 0),
+// so a 256-byte block serves all 128 rows.
+__device__ __forceinline__ uint64_t desc_ones(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)1 << 46);
 }
 
 struct TcParams {
   int N, K, Kpad, ntiles, upb, total_units;
-  uint32_t idesc;
+  uint32_t idesc, idesc_bias;
   int is_bf16;
   uint32_t dyn_bytes;
-  const float *bias;  // -|c|^2/2 per centroid, -inf in the padding
   int32_t *labels;
   float *mindist;
   DevCtl ctl;
@@ -133,18 +165,27 @@ struct Best {
   uint32_t cand[32];  // the chunk that first reached `score`
 };
 
-// Fold one 32-column chunk (first column `col`) into the running arg-max.
-// The candidate copy is written as x + 0 (add.rn.f32), which runs on the
-// full-rate FMA pipe instead of the half-rate integer/logic pipe that the
-// max tree already saturates; it keeps every value but turns -0 into +0,
-// which compares equal, so the index search below finds the same column.
+// (d0, d1) = (a0 + b0, a1 + b1) in one packed fp32 add (FMA pipe).
+__device__ __forceinline__ void add2(uint32_t &d0, uint32_t &d1, uint32_t a0, uint32_t a1, uint32_t b0,
+                                     uint32_t b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\t"
+      "add.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "=r"(d0), "=r"(d1)
+      : "r"(a0), "r"(a1), "r"(b0), "r"(b1));
+}
+
+// Fold one 32-column chunk of scores (first column `col`) into the running
+// arg-max.  The candidate copy is written as x + 0 (packed add.rn.f32x2, two
+// values per instruction on the FMA pipe, leaving the half-rate logic pipe
+// to the max trees); it keeps every value but turns -0 into +0, which
+// compares equal, so the index search below finds the same column.
 __device__ __forceinline__ void fold_chunk(Best &bs, const uint32_t (&v)[32], int col) {
   const float m = max32(v);
   const bool imp = m > bs.score;  // strict: an earlier column keeps a tie
   if (__any_sync(0xffffffffu, imp)) {
     if (imp) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) bs.cand[i] = __float_as_uint(__fadd_rn(__uint_as_float(v[i]), 0.f));
+      for (int i = 0; i < 32; i += 2) add2(bs.cand[i], bs.cand[i + 1], v[i], v[i + 1], 0u, 0u);
       bs.score = m;
       bs.base = col;
     }
@@ -154,9 +195,9 @@ __device__ __forceinline__ void fold_chunk(Best &bs, const uint32_t (&v)[32], in
 template <int KB>
 __global__ void __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
-                     const TcParams p) {
+                     const __grid_constant__ CUtensorMap bmap, const TcParams p) {
   using Cfg = TcCfg<KB>;
-  constexpr int NST = Cfg::NST, XBUF = Cfg::XBUF;
+  constexpr int NST = Cfg::NSLOT, XBUF = Cfg::XBUF;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
 
   const uint32_t rank = cluster_rank();
@@ -174,13 +215,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sX = raw + pad;
   const uint32_t sC = sX + Cfg::X_BYTES;
   float4 *xchg = reinterpret_cast<float4 *>(sm + Cfg::X_BYTES + Cfg::C_BYTES);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Cfg::X_BYTES + Cfg::C_BYTES + Cfg::XCHG_BYTES);
+  float *ones = reinterpret_cast<float *>(sm + Cfg::X_BYTES + Cfg::C_BYTES + Cfg::XCHG_BYTES);
+  uint64_t *bars =
+      reinterpret_cast<uint64_t *>(sm + Cfg::X_BYTES + Cfg::C_BYTES + Cfg::XCHG_BYTES + kOnesBytes);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::NBAR);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };                                   // leader's
   auto empty = [&](int s) { return bar0 + 8u * (NST + s); };                          // each CTA
+  auto slot_c = [&](int s, int kb) { return sC + s * Cfg::SLOT + kb * kStageBytes; };
+  auto slot_bias = [&](int s) { return sC + s * Cfg::SLOT + KB * kStageBytes; };
   auto xfull = [&](int x) { return bar0 + 8u * (2 * NST + x); };                      // leader's
   auto xempty = [&](int x) { return bar0 + 8u * (2 * NST + XBUF + x); };              // each CTA
   auto accfull = [&](int a) { return bar0 + 8u * (2 * NST + 2 * XBUF + a); };         // each CTA
@@ -193,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(full(s), 1);   // the leader's expect_tx; bytes from both CTAs
-      mbar_init(empty(s), 1);  // the epilogue, once the tile using the stage is complete
+      mbar_init(empty(s), 1);  // the epilogue, once the tile using the slot is complete
     }
     for (int x = 0; x < XBUF; ++x) {
       mbar_init(xfull(x), 1);
@@ -212,7 +257,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&xmap);
     tma_prefetch_desc(&cmap);
+    tma_prefetch_desc(&bmap);
   }
+  // The A operand of the bias step: 8 rows of (1, 1, 1, 0 | 0, 0, 0, 0) as
+  // two no-swizzle core matrices (columns 0-3, then 4-7 at +128 B).
+  if (threadIdx.x < kOnesBytes / 4) ones[threadIdx.x] = (threadIdx.x < 32 && (threadIdx.x & 3) < 3) ? 1.f : 0.f;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
   if (warp == kMmaWarp) {
     tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish_pair();
@@ -237,13 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = true;
         if (++xb == XBUF) { xb = 0; xph ^= 1u; }
         for (int j = 0; ok && j < p.ntiles; ++j) {
-          for (int kb = 0; kb < KB; ++kb) {
-            if (!(ok = mbar_wait(empty(st), sph ^ 1u, abort_flag, p.ctl))) break;
-            if (leader) mbar_arrive_expect_tx(full(st), 2 * kStageBytes);
-            tma_load_3d_pair(sC + st * kStageBytes, &cmap, map_to_cta(full(st), 0), kb * kBlkK,
-                             j * kTileN + (int)rank * kHalfN, b);
-            if (++st == NST) { st = 0; sph ^= 1u; }
-          }
+          if (!(ok = mbar_wait(empty(st), sph ^ 1u, abort_flag, p.ctl))) break;
+          if (leader) mbar_arrive_expect_tx(full(st), 2 * (KB * kStageBytes + kBiasBytes));
+          const uint32_t fbar = map_to_cta(full(st), 0);
+          const int c0 = j * kTileN + (int)rank * kHalfN;
+          for (int kb = 0; kb < KB; ++kb) tma_load_3d_pair(slot_c(st, kb), &cmap, fbar, kb * kBlkK, c0, b);
+          tma_load_3d_pair(slot_bias(st), &bmap, fbar, 0, c0, b);
+          if (++st == NST) { st = 0; sph ^= 1u; }
         }
       }
       // After an abort, give copies already issued time to land in this CTA's
@@ -258,30 +308,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ------------------------------------------------- MMA issuer -----
       uint32_t xb = 0, xph = 0, st = 0, sph = 0;
+      const uint64_t ones_desc = desc_ones(smem_u32(ones));
       int t = 0;  // tile counter: accumulator t % 2, its (t / 2)-th use
       bool ok = true;
       for (int u = pair; ok && u < p.total_units; u += npairs) {
         if (!(ok = mbar_wait(xfull(xb), xph, abort_flag, p.ctl))) break;
         const uint32_t xa = sX + xb * KB * kXBytes;
         for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
-          uint32_t stg[KB];
-          for (int kb = 0; kb < KB; ++kb) {
-            stg[kb] = st;
-            if (!(ok = mbar_wait(full(st), sph, abort_flag, p.ctl))) break;
-            if (++st == NST) { st = 0; sph ^= 1u; }
-          }
-          if (!ok) break;
+          const int sl = st;
+          if (!(ok = mbar_wait(full(st), sph, abort_flag, p.ctl))) break;
+          if (++st == NST) { st = 0; sph ^= 1u; }
           const int a = t & 1;
-          // the accumulator was drained and re-armed with this tile's bias
+          // every epilogue warp of the pair has read the accumulator's last tile
           if (!(ok = mbar_wait(accempty(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
           tc_fence_after();
+          const uint32_t acc = tbase + a * kTileN;
+          // accumulator = 1*hi + 1*mid + 1*lo = -|c|^2/2 (overwrites)
+          tc_mma_tf32_pair(acc, ones_desc, desc_kmajor_sw32(slot_bias(sl)), p.idesc_bias, 0u);
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
             const uint64_t ad = desc_kmajor_sw128(xa + kb * kXBytes);
-            const uint64_t bd = desc_kmajor_sw128(sC + stg[kb] * kStageBytes);
+            const uint64_t bd = desc_kmajor_sw128(slot_c(sl, kb));
 #pragma unroll
-            for (int k = 0; k < kBlkK / 16; ++k)
-              tc_mma_f16_pair(tbase + a * kTileN, ad + 2 * k, bd + 2 * k, p.idesc, 1u);
+            for (int k = 0; k < kBlkK / 16; ++k) tc_mma_f16_pair(acc, ad + 2 * k, bd + 2 * k, p.idesc, 1u);
           }
           tc_commit_pair(accfull(a), kBothCtas);
         }
@@ -303,36 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) mbar_arrive(accempty(a));
       else mbar_arrive_cluster_relaxed(map_to_cta(accempty(a), 0));
     };
-    // Walks the pair's tiles in order and yields the bias of this warp's 128
-    // columns of each (null past the last unit).
-    struct BiasIter {
-      const float *row;  // bias of the current unit's problem, this warp's half
-      int u, j;
-    } bi_ = {nullptr, pair, 0};
-    auto bias_row = [&](int u) { return p.bias + (size_t)(u / p.upb) * p.Kpad + h * kHalfN; };
-    bi_.row = bias_row(pair);
-    auto next_bias = [&]() -> const float * {
-      const float *r = bi_.u < p.total_units ? bi_.row + bi_.j * kTileN : nullptr;
-      if (++bi_.j == p.ntiles) {
-        bi_.j = 0;
-        bi_.u += npairs;
-        if (bi_.u < p.total_units) bi_.row = bias_row(bi_.u);
-      }
-      return r;
-    };
-    // Arm both accumulators with the bias of tiles 0 and 1.
-#pragma unroll 1
-    for (int a = 0; a < kAcc; ++a) {
-      if (const float *bp = next_bias()) {
-#pragma unroll 1
-        for (int c = 0; c < kHalfN / 32; ++c) {
-          uint32_t w[32];
-          load_bias32(bp + c * 32, w);
-          FK_TMEM_ST32(t_row + a * kTileN + c * 32, w);
-        }
-      }
-    }
-    tmem_wait_st();
+    // Both accumulators start out free.
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
@@ -353,48 +373,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
       for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
         const int a = t & 1;
-        const float *nbp = next_bias();  // tile t + 2: the next one for this accumulator
         if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
         tc_fence_after();
-        if (h == 0 && q == 0 && lane == 0) {  // the MMA has consumed this tile's centroid stages
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb) mbar_arrive(empty((t * KB + kb) % NST));
-        }
+        if (h == 0 && q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
         const uint32_t ta = t_row + a * kTileN;
         const int col = j * kTileN + h * kHalfN;
-        uint32_t va[32], vb[32], w[32];
-        if (nbp) load_bias32(nbp, w);
+        uint32_t va[32], vb[32];
+        // chunks 0 and 1
         FK_TMEM_LD32(ta, va);
-        FK_TMEM_WAIT_LD(va);
-        // chunk c is reduced while chunk c + 1 is on its way from TMEM; the
-        // next tile's bias goes where chunk c was read
         FK_TMEM_LD32(ta + 32, vb);
-        fold_chunk(bs, va, col);
-        if (nbp) {
-          FK_TMEM_ST32(ta, w);
-          load_bias32(nbp + 32, w);
-        }
-        FK_TMEM_WAIT_LD(vb);
-        FK_TMEM_LD32(ta + 64, va);
-        fold_chunk(bs, vb, col + 32);
-        if (nbp) {
-          FK_TMEM_ST32(ta + 32, w);
-          load_bias32(nbp + 64, w);
-        }
         FK_TMEM_WAIT_LD(va);
-        FK_TMEM_LD32(ta + 96, vb);
-        fold_chunk(bs, va, col + 64);
-        if (nbp) {
-          FK_TMEM_ST32(ta + 64, w);
-          load_bias32(nbp + 96, w);
-        }
         FK_TMEM_WAIT_LD(vb);
-        fold_chunk(bs, vb, col + 96);
-        if (nbp) FK_TMEM_ST32(ta + 96, w);
-        tmem_wait_st();
+        fold_chunk(bs, va, col);
+        fold_chunk(bs, vb, col + 32);
+        // chunks 2 and 3: once they are in registers the accumulator is free
+        FK_TMEM_LD32(ta + 64, va);
+        FK_TMEM_LD32(ta + 96, vb);
+        FK_TMEM_WAIT_LD(va);
+        FK_TMEM_WAIT_LD(vb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(a);
+        fold_chunk(bs, va, col + 64);
+        fold_chunk(bs, vb, col + 96);
       }
       if (!ok) break;
       // lowest column of the candidate chunk holding the maximum
@@ -506,6 +507,21 @@ static bool encode_3d(CUtensorMap *m, DType dt, const void *ptr, int D, int rows
   return r == CUDA_SUCCESS;
 }
 
+// The prepared bias as B x Kpad rows of kBiasTerms fp32 terms, loaded half a
+// tile (128 rows of 32 bytes) at a time with the 32-byte swizzle.
+static bool encode_bias_3d(CUtensorMap *m, const float *bias, int Kpad, int B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kBiasTerms, (cuuint64_t)Kpad, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)kBiasRow, (cuuint64_t)kBiasRow * (cuuint64_t)Kpad};
+  const cuuint32_t box[3] = {(cuuint32_t)kBiasTerms, (cuuint32_t)kHalfN, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(bias), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool tc_shape_ok(DType dt, int D) { return dt != kF32 && D % 8 == 0 && D >= 8 && D <= 128; }
 
 bool tc_aligned(const void *X, const void *C) {
@@ -513,8 +529,8 @@ bool tc_aligned(const void *X, const void *C) {
 }
 
 template <int KB>
-static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, TcParams p, int num_sms,
-                             cudaStream_t s) {
+static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, TcParams p,
+                             int num_sms, cudaStream_t s) {
   static int configured[64] = {};
   static std::mutex mu;
   int dev = 0;
@@ -546,7 +562,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, TcPar
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB>, xm, cm, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB>, xm, cm, bm, p);
   count_launches(1);
   return e;
 }
@@ -554,9 +570,10 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, TcPar
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
                              int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
                              int num_sms, cudaStream_t s) {
-  if (!tc_shape_ok(dt, D) || !tc_aligned(X, C)) return cudaErrorNotSupported;
-  CUtensorMap xm, cm;
-  if (!encode_3d(&xm, dt, X, D, N, B, kRows) || !encode_3d(&cm, dt, C, D, K, B, kHalfN))
+  if (!tc_shape_ok(dt, D) || !tc_aligned(X, C) || (uintptr_t)bias % 16 != 0) return cudaErrorNotSupported;
+  CUtensorMap xm, cm, bm;
+  if (!encode_3d(&xm, dt, X, D, N, B, kRows) || !encode_3d(&cm, dt, C, D, K, B, kHalfN) ||
+      !encode_bias_3d(&bm, bias, Kpad, B))
     return cudaErrorNotSupported;
   TcParams p;
   p.N = N;
@@ -566,8 +583,8 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   p.upb = (N + kRowsUnit - 1) / kRowsUnit;
   p.total_units = p.upb * B;
   p.idesc = idesc_f16(dt == kBF16 ? 1 : 0, kRowsUnit, kTileN);
+  p.idesc_bias = idesc_tf32(kRowsUnit, kTileN);
   p.is_bf16 = dt == kBF16;
-  p.bias = bias;
   p.labels = labels;
   p.mindist = mindist;
   p.ctl = ctl;
@@ -575,8 +592,8 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   if (p.total_units == 0) return cudaSuccess;
   if (Kpad < p.ntiles * kTileN) return cudaErrorInvalidValue;  // the bias must cover every tile
   const int KB = (D + kBlkK - 1) / kBlkK;
-  if (KB == 1) return launch_kb<1>(xm, cm, p, num_sms, s);
-  return launch_kb<2>(xm, cm, p, num_sms, s);
+  if (KB == 1) return launch_kb<1>(xm, cm, bm, p, num_sms, s);
+  return launch_kb<2>(xm, cm, bm, p, num_sms, s);
 }
 
 }  // namespace fk

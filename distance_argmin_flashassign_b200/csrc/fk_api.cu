@@ -137,14 +137,15 @@ static int choose_path(DType dt, int D) {
   return tc_shape_ok(dt, D) ? 1 : 2;
 }
 
-// Assignment of B problems.  cn (the B*Kpad bias -|c|^2/2 of C) may be null,
-// in which case the tensor path computes it into scratch at `cn_ws`.
+// Assignment of B problems.  cn (the prepared bias of C: kBiasTerms floats per
+// padded centroid) may be null, in which case the tensor path computes it into
+// scratch at `cn_ws`.
 static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
                             const float *cn, float *cn_ws, int32_t *labels, float *mindist,
                             cudaStream_t s) {
   const int path = choose_path(dt, D);
   if (path < 0) return fail(FK_ERR_UNSUPPORTED, "tensor-core path forced for an unsupported shape");
-  if (path == 1 && tc_aligned(X, C)) {
+  if (path == 1 && tc_aligned(X, C) && (!cn || (uintptr_t)cn % 16 == 0)) {
     const int Kpad = pad_k(K);
     if (!cn) {
       cudaError_t e = launch_bias(dt, C, B, K, Kpad, D, cn_ws, s);
@@ -157,7 +158,7 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
     cudaGetLastError();
     if (g_assign_path.load() == 1) return fail(FK_ERR_UNSUPPORTED, "tensor maps could not be encoded");
   } else if (path == 1 && g_assign_path.load() == 1) {
-    return fail(FK_ERR_UNSUPPORTED, "tensor-core path needs 16-byte aligned X and C");
+    return fail(FK_ERR_UNSUPPORTED, "tensor-core path needs 16-byte aligned X, C and bias");
   }
   cudaError_t e = launch_assign_simt(dt, X, C, B, N, D, K, labels, mindist, s);
   if (e != cudaSuccess) return cuda_fail(e, "CUDA-core assign kernel");
@@ -215,7 +216,7 @@ fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dtype dt,
   if ((st = device_state(&d)) != FK_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   void *ws = nullptr;
-  if ((st = scratch(*d, s, al256((size_t)B * pad_k(K) * 4), &ws)) != FK_OK) return st;
+  if ((st = scratch(*d, s, al256(bias_bytes(B, K)), &ws)) != FK_OK) return st;
   return run_assign(*d, (DType)dt, X, B, (int)N, D, C, K, nullptr, (float *)ws, labels, mindist, s);
 }
 
@@ -226,7 +227,7 @@ fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C,
 
 int64_t fk_bias_len(int B, int K) {
   if (B < 1 || K < 1) return 0;
-  return (int64_t)B * pad_k(K);
+  return (int64_t)B * pad_k(K) * kBiasTerms;
 }
 
 fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt, float *bias,
@@ -312,7 +313,7 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   const DType t = (DType)dt;
   const int Kpad = pad_k(K);
   const size_t upd = al256(update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D));
-  const size_t cnb = al256((size_t)B * Kpad * 4);
+  const size_t cnb = al256(bias_bytes(B, K));
   const size_t cdb = t == kF32 ? 0 : al256((size_t)B * K * D * dtype_size(t));
   void *ws = nullptr;
   if ((st = scratch(*d, s, upd + cnb + cdb, &ws)) != FK_OK) return st;
@@ -373,7 +374,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   // device buffers, carved from the scratch cache of (device, stream)
   const size_t b_ring = al256((size_t)rows * D * es), b_lab = al256((size_t)rows * 4);
   const size_t b_c32 = al256((size_t)K * D * 4), b_cdt = t == kF32 ? 0 : al256((size_t)K * D * es);
-  const size_t b_cn = al256((size_t)Kpad * 4), b_acc = al256((size_t)K * D * 8);
+  const size_t b_cn = al256(bias_bytes(1, K)), b_acc = al256((size_t)K * D * 8);
   const size_t b_cnt = al256((size_t)K * 8), b_counts = al256((size_t)K * 4);
   const size_t b_upd = al256(update_workspace_bytes(rows, K, D));
   const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd;

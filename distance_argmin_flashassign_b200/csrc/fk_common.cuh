@@ -80,6 +80,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but a thread whose phase is not complete is suspended until
+// it completes or `sleep_ns` nanoseconds pass (the suspend-time hint).  A
+// waiting thread that polls without it keeps issuing instructions and takes
+// issue slots from the warps doing the work on its SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(sleep_ns)
+      : "memory");
+  return ok != 0;
+}
+// Longest single suspension of a waiting thread: the abort flag and the
+// timeout are checked at least this often.
+constexpr uint32_t kWaitSleepNs = 1000000u;
+
 // Wait until the phase of parity `parity` of barrier `bar` has completed.
 // Gives up (returns false) when *abort becomes non-zero or when the wait has
 // lasted longer than ctl.timeout_ns; in the latter case it raises *abort and
@@ -88,15 +106,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           const DevCtl &ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 15) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > ctl.timeout_ns) {
-        *abort = 1;
-        record_status(ctl.status, kStTimeout);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > ctl.timeout_ns) {
+      *abort = 1;
+      record_status(ctl.status, kStTimeout);
+      return false;
     }
   }
 }
@@ -104,7 +120,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Same, bounded by `ns` only (used while draining after an abort).
 __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t ns) {
   const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
     if (globaltimer() - t0 > ns) return false;
   }
   return true;

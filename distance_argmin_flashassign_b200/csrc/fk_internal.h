@@ -17,6 +17,11 @@ int record_error(int status, const char *msg);
 
 constexpr int kCentroidPad = 256;  // centroid tile of the tensor-core kernel
 inline int pad_k(int K) { return (K + kCentroidPad - 1) / kCentroidPad * kCentroidPad; }
+// Floats of prepared bias per (padded) centroid: three tf32-exact terms of
+// -|c|^2/2, then zeros, one 32-byte row per centroid (the K = 8 operand of a
+// tf32 MMA step).
+constexpr int kBiasTerms = 8;
+inline size_t bias_bytes(int B, int K) { return (size_t)B * pad_k(K) * kBiasTerms * sizeof(float); }
 inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
 
 // ---- prep.cu: centroid bias (row norms of the assignment stage) -----------

@@ -8,9 +8,38 @@
 // the tensor cores see them (already rounded to the input type) and padded
 // with -inf up to a multiple of the 256-centroid tile, so padded columns
 // never win.
+//
+// The tensor cores add the bias themselves (one tf32 MMA step against a
+// block of ones starts every tile), so each centroid's bias is stored as
+// kBiasTerms floats: three terms that tf32 represents exactly and whose sum
+// is the fp32 bias, then zeros.
 #include "fk_internal.h"
 
 namespace fk {
+
+// Keep the 11 leading significand bits (sign, exponent and 10 fraction bits):
+// the value a tf32 operand holds exactly.
+__device__ __forceinline__ float tf32_head(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
+
+// Terms of the bias s at dst[0..kBiasTerms): hi + mid + lo == s exactly.
+// hi keeps s's top 11 significand bits; s - hi is exact (same sign and
+// binade) and has at most 13 significant bits, of which mid keeps the top 11
+// and lo = (s - hi) - mid the last 2, again exactly.
+__device__ __forceinline__ void store_bias_terms(float *dst, float s) {
+  const float hi = tf32_head(s);
+  const float r1 = s - hi;
+  const float mid = tf32_head(r1);
+  dst[0] = hi;
+  dst[1] = mid;
+  dst[2] = r1 - mid;
+#pragma unroll
+  for (int i = 3; i < kBiasTerms; ++i) dst[i] = 0.f;
+}
+__device__ __forceinline__ void store_bias_padding(float *dst) {
+  dst[0] = __int_as_float(0xff800000);  // -inf: a padded column never wins
+#pragma unroll
+  for (int i = 1; i < kBiasTerms; ++i) dst[i] = 0.f;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(256) bias_kernel(const T *__restrict__ C, int B, int K, int Kpad,
@@ -21,7 +50,7 @@ __global__ void __launch_bounds__(256) bias_kernel(const T *__restrict__ C, int 
        r += (long long)gridDim.x * 8) {
     const int b = (int)(r / Kpad), j = (int)(r % Kpad);
     if (j >= K) {
-      if (lane == 0) bias[r] = __int_as_float(0xff800000);
+      if (lane == 0) store_bias_padding(bias + r * kBiasTerms);
       continue;
     }
     const T *c = C + ((size_t)b * K + j) * D;
@@ -31,7 +60,7 @@ __global__ void __launch_bounds__(256) bias_kernel(const T *__restrict__ C, int 
       s = fmaf(v, v, s);
     }
     s = warp_sum(s);
-    if (lane == 0) bias[r] = -0.5f * s;
+    if (lane == 0) store_bias_terms(bias + r * kBiasTerms, -0.5f * s);
   }
 }
 
@@ -45,7 +74,7 @@ __global__ void __launch_bounds__(256) round_bias_kernel(const float *__restrict
        r += (long long)gridDim.x * 8) {
     const int b = (int)(r / Kpad), j = (int)(r % Kpad);
     if (j >= K) {
-      if (lane == 0) bias[r] = __int_as_float(0xff800000);
+      if (lane == 0) store_bias_padding(bias + r * kBiasTerms);
       continue;
     }
     const size_t off = ((size_t)b * K + j) * D;
@@ -57,7 +86,7 @@ __global__ void __launch_bounds__(256) round_bias_kernel(const float *__restrict
       s = fmaf(v, v, s);
     }
     s = warp_sum(s);
-    if (lane == 0) bias[r] = -0.5f * s;
+    if (lane == 0) store_bias_terms(bias + r * kBiasTerms, -0.5f * s);
   }
 }
 

@@ -112,16 +112,21 @@ FK_API fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dt
 /* ------------------------------------------------------------------------
  * Two-phase assignment for callers that iterate (Lloyd loops, benchmarks).
  *
- * fk_bias_len -- number of floats of the bias buffer for B problems of K
- *   centroids (K rounded up to the 256-centroid tile, per problem).
+ * fk_bias_len -- number of floats of the prepared bias for B problems of K
+ *   centroids: 8 per centroid, K rounded up to the 256-centroid tile, per
+ *   problem.
  * fk_prepare_centroids -- the preparation step of the assignment stage:
  *   C_dt = C32 rounded to dt (round-to-nearest-even; a plain copy for
- *   FK_F32, skipped when C_dt == C32) and bias = -|C_dt[k]|^2 / 2 in fp32,
- *   with -inf in the padding so padded columns never win.  The tensor-core
- *   kernel ranks centroids by <x, c> + bias, which orders them exactly as the
- *   squared distance does.  One kernel.
+ *   FK_F32, skipped when C_dt == C32) and the bias b_k = -|C_dt[k]|^2 / 2,
+ *   computed in fp32.  The tensor-core kernel ranks centroids by
+ *   <x, c> + b, which orders them exactly as the squared distance does; its
+ *   tensor cores add b themselves, so each centroid's bias is stored as a
+ *   32-byte row of 8 floats: three terms that tf32 holds exactly and whose
+ *   sum is b exactly, then five zeros.  Padded centroids get (-inf, 0, ...)
+ *   so they never win.  One kernel.
  *   C32 device B x K x D fp32; C_dt device B x K x D of dt; bias device
- *   fk_bias_len(B, K) floats.
+ *   fk_bias_len(B, K) floats, 16-byte aligned for the tensor-core path (a
+ *   less aligned bias sends fk_assign_prepared to the CUDA-core kernel).
  * fk_assign_prepared -- fk_assign_batched against prepared centroids and
  *   bias; launches exactly one kernel (the CUDA-core kernel, which computes
  *   direct differences, does not read the bias).

@@ -230,6 +230,29 @@ def test_ooc_matches_in_core(dtype):
     assert int(cnt_h.sum()) == N
 
 
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_prepared_bias_is_an_exact_tf32_split(dtype):
+    # Each centroid's prepared bias is 8 floats: three terms that tf32 holds
+    # exactly (low 13 fraction bits zero), summing exactly to one fp32 value
+    # that is -|c_dt|^2/2 up to the rounding of an fp32 sum of D squares;
+    # then zeros.  Padded centroids hold (-inf, 0, ...).
+    B, K, D = 2, 300, 64
+    g = torch.Generator().manual_seed(3)
+    C = torch.randn(B, K, D, generator=g) * torch.logspace(-3, 3, K).view(1, K, 1)
+    C_dt, bias = fk.fk_prepare_centroids(C.to(DEV), dtype)
+    Kpad = (K + 255) // 256 * 256
+    terms = bias.view(B, Kpad, 8).cpu()
+    bits = terms.view(torch.int32)
+    real = terms[:, :K]
+    assert torch.all((bits[:, :K, :3] & 0x1FFF) == 0)
+    assert torch.all(real[..., 3:] == 0)
+    s64 = real[..., :3].double().sum(-1)
+    assert torch.equal(s64.float().double(), s64)  # the terms add up to an fp32 value
+    ref = -0.5 * (C_dt.cpu().double() ** 2).sum(-1)
+    assert torch.all((s64 - ref).abs() <= 2 * D * 2.0**-24 * ref.abs())
+    assert torch.all(torch.isneginf(terms[:, K:, 0])) and torch.all(terms[:, K:, 1:] == 0)
+
+
 def test_ooc_repeated_calls_and_workspace_release():
     # The out-of-core driver keeps its buffers, side stream and events in the
     # scratch cache: repeated calls reuse them, and a call after
