@@ -62,21 +62,23 @@ static SortPlan plan_sort(long long Ntot, long long Ktot) {
   return p;
 }
 
-// Positions per segment-sum warp: enough warps for about one wave of a
-// B200 (148 SMs x 12 resident warps), at least 256.  Depends on Ntot only, so
-// the summation order (and the result) does not depend on the device.
+// Positions per segment-sum worker: enough workers for about one wave of a
+// B200 (148 SMs x 48 resident half-warp workers), at least 128.  Depends on
+// Ntot only, so the summation order (and the result) does not depend on the
+// device.
 static int chunk_rows_R(long long Ntot) {
-  long long R = (Ntot + 1775) / 1776;
+  long long R = (Ntot + 7103) / 7104;
   R = (R + 31) / 32 * 32;
-  return (int)(R < 256 ? 256 : R);
+  return (int)(R < 128 ? 128 : R);
 }
 
 // --------------------------------------------------------------- sorting --
-__device__ __forceinline__ int first_key(const int32_t *__restrict__ labels, int pos, int N, int K,
-                                         int B, int *status) {
-  int lab = labels[pos];
+// Sort key of position pos from its label: b*K + label for problem b.  A
+// label outside [0, K) counts as 0 and sets `bad`; the caller records it
+// once, after all of its loads, so that no atomic sits between them.
+__device__ __forceinline__ int key_of_label(int lab, int pos, int N, int K, int B, bool &bad) {
   if ((unsigned)lab >= (unsigned)K) {
-    record_status(status, kStBadLabel);
+    bad = true;
     lab = 0;
   }
   return B > 1 ? (pos / N) * K + lab : lab;
@@ -90,19 +92,27 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t 
   __shared__ int hist[kMaxBins + 1];
   for (int i = threadIdx.x; i <= nbins; i += kSortThreads) hist[i] = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31;
   const int base = blockIdx.x * kSortTile;
-#pragma unroll 4
+  // all of the thread's keys are loaded before any is counted (16 loads in
+  // flight), then counted with shared-memory atomics
+  int v[kSortItems];
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * kSortThreads + threadIdx.x;
+    v[it] = pos < Ntot ? keys[pos] : 0;
+  }
+  bool bad = false;
+#pragma unroll
   for (int it = 0; it < kSortItems; ++it) {
     const int pos = base + it * kSortThreads + threadIdx.x;
     int d = nbins;  // spare bin for positions past the end
     if (pos < Ntot) {
-      const int key = FIRST ? first_key(keys, pos, N, K, B, status) : keys[pos];
+      const int key = FIRST ? key_of_label(v[it], pos, N, K, B, bad) : v[it];
       d = (key >> shift) & (nbins - 1);
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, d);
-    if (lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+    atomicAdd(&hist[d], 1);
   }
+  if (bad) record_status(status, kStBadLabel);
   __syncthreads();
   for (int i = threadIdx.x; i < nbins; i += kSortThreads) H[(size_t)i * T + blockIdx.x] = hist[i];
 }
@@ -128,17 +138,24 @@ __global__ void __launch_bounds__(256) scan_rows_kernel(int *__restrict__ H, int
   if (lane == 0) totals[w] = carry;
 }
 
+static size_t scatter_smem_bytes(int nbins) {
+  return (size_t)(2 * nbins + 8 + 2 * kSortTile) * 4 + (size_t)kSortWarps * (nbins + 1) * 2;
+}
+
 template <bool FIRST>
 __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in, int32_t *__restrict__ keys_out,
     int32_t *__restrict__ vals_out, int Ntot, int N, int K, int B, int shift, int nbins, int T,
     const int *__restrict__ H, const int *__restrict__ totals, int *status) {
   extern __shared__ int sh[];
-  int *dbase = sh;                                                   // [nbins]
-  int *wsum = sh + nbins;                                            // [8]
-  uint16_t *wcnt = reinterpret_cast<uint16_t *>(sh + nbins + 8);     // [8][nbins + 1]
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int stride = nbins + 1;
+  int *dbase = sh;                                                   // [nbins]
+  int *tstart = sh + nbins;                                          // [nbins]
+  int *wsum = sh + 2 * nbins;                                        // [8]
+  int *keys_s = sh + 2 * nbins + 8;                                  // [kSortTile]
+  int *vals_s = keys_s + kSortTile;                                  // [kSortTile]
+  uint16_t *wcnt = reinterpret_cast<uint16_t *>(vals_s + kSortTile);  // [8][nbins + 1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   // digit base of this tile = exclusive scan of digit totals + tile prefix
   const int per = (nbins + kSortThreads - 1) / kSortThreads;
@@ -171,42 +188,89 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   const int base = blockIdx.x * kSortTile + warp * (kSortItems * 32);
   const unsigned lt_mask = (1u << lane) - 1u;
   uint16_t *mycnt = wcnt + warp * stride;
+  // all of the warp's keys and values are loaded before the ranking starts
 #pragma unroll
   for (int it = 0; it < kSortItems; ++it) {
     const int pos = base + it * 32 + lane;
-    int d = nbins, key = 0, val = 0;
+    keyr[it] = pos < Ntot ? keys_in[pos] : 0;
+    valr[it] = pos < Ntot ? (FIRST ? pos : vals_in[pos]) : 0;
+  }
+  bool bad = false;
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * 32 + lane;
+    int d = nbins;
     if (pos < Ntot) {
-      key = FIRST ? first_key(keys_in, pos, N, K, B, status) : keys_in[pos];
-      val = FIRST ? pos : vals_in[pos];
-      d = (key >> shift) & (nbins - 1);
+      if (FIRST) keyr[it] = key_of_label(keyr[it], pos, N, K, B, bad);
+      d = (keyr[it] >> shift) & (nbins - 1);
     }
     const unsigned peers = __match_any_sync(0xffffffffu, d);
     const int c = mycnt[d];
     __syncwarp();
     if (lane == __ffs(peers) - 1) mycnt[d] = (uint16_t)(c + __popc(peers));
     __syncwarp();
-    keyr[it] = key;
-    valr[it] = val;
     locr[it] = c + __popc(peers & lt_mask);
   }
+  if (bad) record_status(status, kStBadLabel);
   __syncthreads();
-  for (int d = tid; d < nbins; d += kSortThreads) {
+  // per digit: exclusive prefix over warps (in place) and the tile's count,
+  // then the exclusive scan of the tile's counts over digits: where each
+  // digit's run starts in the tile's sorted order
+  int cnt[kMaxBins / kSortThreads];
+  int tsum = 0;
+  for (int i = 0; i < per; ++i) {
+    const int d = tid * per + i;
     int r = 0;
-    for (int w = 0; w < kSortWarps; ++w) {
-      const int t = wcnt[w * stride + d];
-      wcnt[w * stride + d] = (uint16_t)r;
-      r += t;
-    }
+    if (d < nbins)
+      for (int w = 0; w < kSortWarps; ++w) {
+        const int t = wcnt[w * stride + d];
+        wcnt[w * stride + d] = (uint16_t)r;
+        r += t;
+      }
+    cnt[i] = r;
+    tsum += r;
+  }
+  int tincl = tsum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, tincl, o);
+    if (lane >= o) tincl += n;
+  }
+  __syncthreads();  // everyone is done reading wsum (digit bases above)
+  if (lane == 31) wsum[warp] = tincl;
+  __syncthreads();
+  int trun = tincl - tsum;
+  for (int w = 0; w < warp; ++w) trun += wsum[w];
+  for (int i = 0; i < per; ++i) {
+    const int d = tid * per + i;
+    if (d < nbins) tstart[d] = trun;
+    trun += cnt[i];
   }
   __syncthreads();
+  // exchange through shared memory into the tile's sorted order ...
 #pragma unroll
   for (int it = 0; it < kSortItems; ++it) {
     const int pos = base + it * 32 + lane;
     if (pos < Ntot) {
       const int d = (keyr[it] >> shift) & (nbins - 1);
-      const int o = dbase[d] + mycnt[d] + locr[it];
-      keys_out[o] = keyr[it];
-      vals_out[o] = valr[it];
+      const int lp = tstart[d] + mycnt[d] + locr[it];
+      keys_s[lp] = keyr[it];
+      vals_s[lp] = valr[it];
+    }
+  }
+  __syncthreads();
+  // ... and write it out in that order: consecutive threads store
+  // consecutive positions of a digit's run
+  const int nvalid = (Ntot - blockIdx.x * kSortTile) < kSortTile ? (Ntot - blockIdx.x * kSortTile) : kSortTile;
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int idx = it * kSortThreads + tid;
+    if (idx < nvalid) {
+      const int key = keys_s[idx];
+      const int d = (key >> shift) & (nbins - 1);
+      const int o = dbase[d] + (idx - tstart[d]);
+      keys_out[o] = key;
+      vals_out[o] = vals_s[idx];
     }
   }
 }
@@ -520,19 +584,130 @@ __global__ void __launch_bounds__(kSegWarps * 32) segsum_staged_kernel(
   if (p1 == Ntot) write_offsets(off, cur, Ktot, Ntot, lane);
 }
 
-// One block per cluster (grid-stride): counts, then the fixed-order sum of
-// the partials of a segment that crosses chunk borders.
+// Gather workers of W lanes (W = row bytes / 16, 8 to 32): lane l of a
+// worker owns the 16 bytes [16l, 16l + 16) of every row, and every worker
+// sums the rows of its own chunk of R sorted positions, GATHER_ROWS of them
+// in flight at a time (one 16-byte load per lane and row).  Small workers
+// mean many independent gathers per SM, which is what HBM needs to serve
+// random rows at full rate.  The segmentation (which segments are whole,
+// which go to the two partial slots of the chunk) is the one of
+// segsum_kernel, with worker index in place of warp index.
+constexpr int kGatherRows = 8;
+template <typename T, int W, int MODE>
+__global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restrict__ X, int D,
+                                                            const int32_t *__restrict__ perm,
+                                                            const int32_t *__restrict__ skeys, int Ntot, int Ktot,
+                                                            int R, float *__restrict__ C, double *__restrict__ acc,
+                                                            float *__restrict__ parts, int *__restrict__ off) {
+  constexpr int EPL = 16 / (int)sizeof(T);  // elements per lane
+  constexpr int U = kGatherRows;
+  static_assert(W >= U && W <= 32 && (32 % W) == 0, "worker width");
+  const int lw = threadIdx.x % W;
+  const long long wq = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / W;  // worker = chunk index
+  const long long p0l = wq * R;
+  const bool live = p0l < Ntot;
+  const int p0 = live ? (int)p0l : Ntot;
+  const int p1 = (Ntot - p0) < R ? Ntot : p0 + R;
+  int cur = 0, s = p0;
+  bool split_start = false, split_end = false;
+  if (live) {
+    const int kfirst = skeys[p0];
+    const int kprev = p0 > 0 ? skeys[p0 - 1] : -1;
+    split_start = kprev == kfirst;
+    split_end = p1 < Ntot && skeys[p1] == skeys[p1 - 1];
+    for (int kk = kprev + 1 + lw; kk <= kfirst; kk += W) off[kk] = p0;
+    cur = kfirst;
+  }
+  float a[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) a[i] = 0.f;
+  auto flush = [&](int k, int sb, int se) {
+    const bool split = (sb == p0 && split_start) || (se == p1 && split_end);
+    if (!split) {
+      if (MODE == kMean) {
+        const float inv = 1.f / (float)(se - sb);
+        float *dst = C + (size_t)k * D + lw * EPL;
+#pragma unroll
+        for (int i = 0; i < EPL; i += 4)
+          *reinterpret_cast<float4 *>(dst + i) = make_float4(a[i] * inv, a[i + 1] * inv, a[i + 2] * inv, a[i + 3] * inv);
+      } else {
+        double *dst = acc + (size_t)k * D + lw * EPL;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) dst[i] += (double)a[i];
+      }
+    } else {
+      float *dst = parts + ((size_t)wq * 2 + (sb == p0 ? 0 : 1)) * D + lw * EPL;
+#pragma unroll
+      for (int i = 0; i < EPL; i += 4) *reinterpret_cast<float4 *>(dst + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+    }
+  };
+  // every worker of the warp runs the same number of batches (shuffles stay
+  // converged); positions past a worker's end are masked
+  const int nb = (R + U - 1) / U;
+  for (int bt = 0; bt < nb; ++bt) {
+    const int b0 = p0 + bt * U;
+    const int mk = (lw < U && b0 + lw < p1) ? skeys[b0 + lw] : 0;
+    const int mr = (lw < U && b0 + lw < p1) ? perm[b0 + lw] : 0;
+    uint4 v[U];
+    int kk[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int row = __shfl_sync(0xffffffffu, mr, u, W);
+      kk[u] = __shfl_sync(0xffffffffu, mk, u, W);
+      v[u] = (b0 + u < p1) ? __ldg(reinterpret_cast<const uint4 *>(X + (size_t)row * D) + lw) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (b0 + u < p1) {
+        if (kk[u] != cur) {
+          flush(cur, s, b0 + u);
+          for (int q = cur + 1 + lw; q <= kk[u]; q += W) off[q] = b0 + u;
+          cur = kk[u];
+          s = b0 + u;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) a[i] = 0.f;
+        }
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        if constexpr (sizeof(T) == 4) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) a[i] += __uint_as_float(w[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float f[2];
+            if constexpr (std::is_same<T, __nv_bfloat16>::value) unpack_bf162(w[i], f);
+            else unpack_half2(w[i], f);
+            a[2 * i] += f[0];
+            a[2 * i + 1] += f[1];
+          }
+        }
+      }
+    }
+  }
+  if (live) {
+    flush(cur, s, p1);
+    if (p1 == Ntot)
+      for (int q = cur + 1 + lw; q <= Ktot; q += W) off[q] = Ntot;
+  }
+}
+
+// One warp per cluster (grid-stride): the count, then, for a segment that
+// crosses chunk borders but has at most kHotParts partial rows, the sum of
+// those rows in chunk order (two interleaved running sums, added at the end:
+// a fixed order), divided by the count.  Segments inside one chunk were
+// written by their worker; segments with more partial rows (the hot clusters
+// of a skewed distribution) are left to seg_finalize_hot_kernel.
+constexpr int kHotParts = 16;
 template <int MODE>
-__global__ void __launch_bounds__(512) seg_finalize_kernel(const int *__restrict__ off, int Ktot, int D, int R,
+__global__ void __launch_bounds__(256) seg_finalize_kernel(const int *__restrict__ off, int Ktot, int D, int R,
                                                            const float *__restrict__ parts,
                                                            float *__restrict__ C, int32_t *__restrict__ counts,
                                                            double *__restrict__ acc, long long *__restrict__ cnt) {
-  __shared__ float red[512];
-  const int tid = threadIdx.x;
-  const int G = D >= 512 ? 1 : 512 / D;  // groups of partials summed in parallel
-  for (int k = blockIdx.x; k < Ktot; k += gridDim.x) {
+  const int lane = threadIdx.x & 31;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long k = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; k < Ktot; k += nw) {
     const int s = off[k], e = off[k + 1], n = e - s;
-    if (tid == 0) {
+    if (lane == 0) {
       if (MODE == kMean) {
         if (counts) counts[k] = n;
       } else {
@@ -543,30 +718,90 @@ __global__ void __launch_bounds__(512) seg_finalize_kernel(const int *__restrict
     const int q0 = s / R, q1 = (e - 1) / R;
     if (q0 == q1) continue;  // segment inside one chunk: already written
     const int np = q1 - q0 + 1;
+    if (np > kHotParts) continue;
     const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
     auto part_row = [&](int i) { return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D; };
-    if (G > 1) {
-      const int g = tid / D, d = tid % D;
-      float t = 0.f;
-      if (g < G)
-        for (int i = g; i < np; i += G) t += part_row(i)[d];
-      red[tid] = t;
-      __syncthreads();
-      if (tid < D) {
-        float tot = 0.f;
-        for (int gg = 0; gg < G; ++gg) tot += red[gg * D + tid];
-        if (MODE == kMean) C[(size_t)k * D + tid] = tot / (float)n;
-        else acc[(size_t)k * D + tid] += (double)tot;
+    // 4 dimensions per lane per pass; every partial row's loads are
+    // independent of the running sums, so they are all in flight together
+    for (int d0 = 0; d0 < D; d0 += 128) {
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < np; ++i) {
+        const float *row = part_row(i) + d0;
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = d0 + lane + 32 * j < D ? row[lane + 32 * j] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) t[j] += v[j];
       }
-      __syncthreads();
-    } else {
-      for (int d = tid; d < D; d += blockDim.x) {
-        float tot = 0.f;
-        for (int i = 0; i < np; ++i) tot += part_row(i)[d];
-        if (MODE == kMean) C[(size_t)k * D + d] = tot / (float)n;
-        else acc[(size_t)k * D + d] += (double)tot;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = d0 + lane + 32 * j;
+        if (d >= D) continue;
+        if (MODE == kMean) C[(size_t)k * D + d] = t[j] / (float)n;
+        else acc[(size_t)k * D + d] += (double)t[j];
       }
     }
+  }
+}
+
+// Segments with more than kHotParts partial rows.  Block b owns the clusters
+// b, b + G, b + 2G, ... (G blocks; hot clusters of a skewed distribution are
+// usually consecutive ids, so they land in different blocks).  It looks at
+// 1024 of them at once (one per thread), lists the hot ones in shared
+// memory, then gives each of them all of its 32 warps: warp w sums
+// the partial rows w, w + 32, ... (lanes over dimensions), then thread d adds
+// the 32 warp sums of dimension d in warp order: a fixed order.
+template <int MODE>
+__global__ void __launch_bounds__(1024) seg_finalize_hot_kernel(const int *__restrict__ off, int Ktot, int D, int R,
+                                                                const float *__restrict__ parts,
+                                                                float *__restrict__ C, double *__restrict__ acc) {
+  __shared__ float red[32][129];
+  __shared__ int hot[1024];
+  __shared__ int nhot;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long G = gridDim.x;
+  for (long long i0 = 0; blockIdx.x + G * i0 < Ktot; i0 += 1024) {
+    if (threadIdx.x == 0) nhot = 0;
+    __syncthreads();
+    {
+      const long long kl = blockIdx.x + G * (i0 + threadIdx.x);
+      const int k = (int)kl;
+      if (kl < Ktot) {
+        const int s = off[k], e = off[k + 1];
+        if (e > s && (e - 1) / R - s / R + 1 > kHotParts) hot[atomicAdd(&nhot, 1)] = k;
+      }
+    }
+    __syncthreads();
+    const int nh = nhot;
+    for (int h = 0; h < nh; ++h) {
+    const int k = hot[h];
+    const int s = off[k], e = off[k + 1], n = e - s;
+    const int q0 = s / R, q1 = (e - 1) / R;
+    const int np = q1 - q0 + 1;
+    const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
+    auto part_row = [&](int i) { return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D; };
+    for (int d0 = 0; d0 < D; d0 += 128) {
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = w; i < np; i += 32) {
+        const float *row = part_row(i) + d0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (d0 + lane + 32 * j < D) t[j] += row[lane + 32 * j];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) red[w][lane + 32 * j] = t[j];
+      __syncthreads();
+      if (threadIdx.x < 128 && d0 + threadIdx.x < D) {
+        float tot = 0.f;
+        for (int ww = 0; ww < 32; ++ww) tot += red[ww][threadIdx.x];
+        const size_t o = (size_t)k * D + d0 + threadIdx.x;
+        if (MODE == kMean) C[o] = tot / (float)n;
+        else acc[o] += (double)tot;
+      }
+      __syncthreads();
+    }
+    }
+    __syncthreads();  // the list is rebuilt for the next window
   }
 }
 
@@ -643,6 +878,20 @@ static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_
   const bool aligned = ((uintptr_t)a.X % 16 == 0);
   const int nacc_c = D % 32 == 0 ? D / 32 : 0;
   const int rb = nacc_c * (int)sizeof(T) * 32;
+  {
+    const int W = D * (int)sizeof(T) / 16;
+    const long long nworkers = ((long long)Ntot + R - 1) / R;
+    if (aligned && (D * (int)sizeof(T)) % 16 == 0 && (W == 8 || W == 16 || W == 32)) {
+      const int ggrid = (int)((nworkers * W + 255) / 256);
+#define FK_GATHER(WW)                                                                                 \
+  return (void)segsum_gather_kernel<T, WW, MODE><<<ggrid, 256, 0, s>>>(X, D, perm, skeys, Ntot, Ktot, R, a.C, \
+                                                                       a.acc, parts, off)
+      if (W == 8) FK_GATHER(8);
+      if (W == 16) FK_GATHER(16);
+      FK_GATHER(32);
+#undef FK_GATHER
+    }
+  }
   if (aligned && rb % 16 == 0 && rb > 0 && rb <= 512) {
     if (nacc_c == 1) return launch_staged<T, MODE, 1>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
     if (nacc_c == 2) return launch_staged<T, MODE, 2>(a, perm, skeys, Ntot, Ktot, R, parts, off, s);
@@ -680,6 +929,17 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
   const int N = (int)Ntot;
   int nl = 0;
 
+  {  // the scatter's tile exchange needs more than the default 48 KB of shared memory
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !configured[dev]) {
+      const int most = (int)scatter_smem_bytes(kMaxBins);
+      cudaFuncSetAttribute(radix_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(radix_scatter_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      configured[dev] = true;
+    }
+  }
   const int32_t *kin = a.labels, *vin = nullptr;
   int32_t *kout = w.kA, *vout = w.vA;
   for (int pass = 0; pass < sp.npass; ++pass) {
@@ -691,7 +951,7 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
       radix_hist_kernel<false><<<sp.T, kSortThreads, 0, s>>>(kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
                                                              sp.T, w.H, ctl.status);
     scan_rows_kernel<<<(nbins + 7) / 8, 256, 0, s>>>(w.H, sp.T, nbins, w.totals);
-    const size_t shb = (size_t)(nbins + 8) * 4 + (size_t)kSortWarps * (nbins + 1) * 2;
+    const size_t shb = scatter_smem_bytes(nbins);
     if (pass == 0)
       radix_scatter_kernel<true><<<sp.T, kSortThreads, shb, s>>>(kin, vin, kout, vout, N, a.N, a.K, a.B,
                                                                  sp.shift[pass], nbins, sp.T, w.H,
@@ -722,14 +982,19 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
       a.mode == kMean ? launch_segsum<__nv_bfloat16, kMean>(a, perm, skeys, N, KT, R, w.parts, w.off, s)
                       : launch_segsum<__nv_bfloat16, kAccumulate>(a, perm, skeys, N, KT, R, w.parts, w.off, s);
   }
-  const int fgrid = (int)(Ktot < (long long)num_sms * 4 ? Ktot : (long long)num_sms * 4);
-  if (a.mode == kMean)
-    seg_finalize_kernel<kMean><<<fgrid, 512, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
+  const long long fwarps = Ktot < (long long)num_sms * 64 ? Ktot : (long long)num_sms * 64;
+  const int fgrid = (int)((fwarps + 7) / 8);
+  const int hgrid = (int)(Ktot < (long long)num_sms ? Ktot : (long long)num_sms);
+  if (a.mode == kMean) {
+    seg_finalize_kernel<kMean><<<fgrid, 256, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
                                                      nullptr, nullptr);
-  else
-    seg_finalize_kernel<kAccumulate><<<fgrid, 512, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr,
+    seg_finalize_hot_kernel<kMean><<<hgrid, 1024, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, nullptr);
+  } else {
+    seg_finalize_kernel<kAccumulate><<<fgrid, 256, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr,
                                                            nullptr, a.acc, a.cnt);
-  nl += 2;
+    seg_finalize_hot_kernel<kAccumulate><<<hgrid, 1024, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr, a.acc);
+  }
+  nl += 3;
   count_launches(nl);
   return cudaGetLastError();
 }
