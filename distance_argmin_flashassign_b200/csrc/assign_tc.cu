@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------ TMA producer ----
       uint32_t xb = 0, xph = 0, st = 0, sph = 0;
-      bool ok = true, issued = false;
+      bool ok = true, issued = false, waited = false;
       for (int u = pair; ok && u < p.total_units; u += npairs) {
         const int b = u / p.upb, r0 = (u % p.upb) * kRowsUnit + (int)rank * kRows;
         if (!(ok = mbar_wait(xempty(xb), xph ^ 1u, abort_flag, p.ctl))) break;
@@ -286,6 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d_pair(sX + (xb * KB + kb) * kXBytes, &xmap, xbar, kb * kBlkK, r0, b);
         issued = true;
         if (++xb == XBUF) { xb = 0; xph ^= 1u; }
+        if (!waited) {
+          // The kernel may be launched before the one that prepared the
+          // centroids and the bias has finished (programmatic stream
+          // serialization): X is input only and loads at once, the centroid
+          // tiles wait until that kernel's writes are visible.
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          waited = true;
+        }
         for (int j = 0; ok && j < p.ntiles; ++j) {
           if (!(ok = mbar_wait(empty(st), sph ^ 1u, abort_flag, p.ctl))) break;
           if (leader) mbar_arrive_expect_tx(full(st), 2 * (KB * kStageBytes + kBiasBytes));
@@ -555,13 +563,17 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = dyn;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // may start while the previous kernel in the stream drains; the producer
+  // waits for it before the first centroid load (see the kernel)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB>, xm, cm, bm, p);
   count_launches(1);
   return e;

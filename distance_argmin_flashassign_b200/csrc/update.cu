@@ -27,6 +27,29 @@
 
 namespace fk {
 
+// Kernels of the update are launched with programmatic stream serialization:
+// a kernel may start (set up shared memory, compute addresses) while the one
+// before it drains, and waits here before its first read of that kernel's
+// results.  The wait returns once the previous grid has completed and its
+// writes are visible.
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kSortThreads = 256;
 constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortThreads * kSortItems;  // 4096 keys per tile
@@ -92,6 +115,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t 
   __shared__ int hist[kMaxBins + 1];
   for (int i = threadIdx.x; i <= nbins; i += kSortThreads) hist[i] = 0;
   __syncthreads();
+  wait_prior_grid();
   const int base = blockIdx.x * kSortTile;
   // all of the thread's keys are loaded before any is counted (16 loads in
   // flight), then counted with shared-memory atomics
@@ -121,6 +145,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t 
 __global__ void __launch_bounds__(256) scan_rows_kernel(int *__restrict__ H, int T, int nbins,
                                                         int *__restrict__ totals) {
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  wait_prior_grid();
   if (w >= nbins) return;
   int *row = H + (size_t)w * T;
   int carry = 0;
@@ -156,6 +181,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   int *vals_s = keys_s + kSortTile;                                  // [kSortTile]
   uint16_t *wcnt = reinterpret_cast<uint16_t *>(vals_s + kSortTile);  // [8][nbins + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  wait_prior_grid();
 
   // digit base of this tile = exclusive scan of digit totals + tile prefix
   const int per = (nbins + kSortThreads - 1) / kSortThreads;
@@ -381,6 +407,7 @@ __global__ void __launch_bounds__(256) segsum_kernel(const T *__restrict__ X, in
                                                      float *__restrict__ parts, int *__restrict__ off) {
   constexpr int PF = NACC <= 4 ? 8 : (NACC <= 8 ? 4 : (NACC <= 16 ? 2 : 1));  // rows in flight
   const int lane = threadIdx.x & 31;
+  wait_prior_grid();
   const long long wq = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long p0l = wq * R;
   if (p0l >= Ntot) return;
@@ -488,6 +515,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) segsum_staged_kernel(
   static_assert(RB % 16 == 0, "rows must be whole 16-byte pieces");
   extern __shared__ __align__(16) uint8_t seg_smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  wait_prior_grid();
   uint8_t *ring = seg_smem + wib * (kSegStages * SLOT);
   const long long wq = (long long)blockIdx.x * kSegWarps + wib;
   const long long p0l = wq * R;
@@ -604,6 +632,7 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
   static_assert(W >= U && W <= 32 && (32 % W) == 0, "worker width");
   const int lw = threadIdx.x % W;
   const long long wq = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / W;  // worker = chunk index
+  wait_prior_grid();
   const long long p0l = wq * R;
   const bool live = p0l < Ntot;
   const int p0 = live ? (int)p0l : Ntot;
@@ -705,6 +734,7 @@ __global__ void __launch_bounds__(256) seg_finalize_kernel(const int *__restrict
                                                            double *__restrict__ acc, long long *__restrict__ cnt) {
   const int lane = threadIdx.x & 31;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  wait_prior_grid();
   for (long long k = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; k < Ktot; k += nw) {
     const int s = off[k], e = off[k + 1], n = e - s;
     if (lane == 0) {
@@ -759,6 +789,7 @@ __global__ void __launch_bounds__(1024) seg_finalize_hot_kernel(const int *__res
   __shared__ int hot[1024];
   __shared__ int nhot;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  wait_prior_grid();
   const long long G = gridDim.x;
   for (long long i0 = 0; blockIdx.x + G * i0 < Ktot; i0 += 1024) {
     if (threadIdx.x == 0) nhot = 0;
@@ -809,6 +840,7 @@ __global__ void __launch_bounds__(256) divide_acc_kernel(const double *__restric
                                                          const long long *__restrict__ cnt, int Ktot, int D,
                                                          float *__restrict__ C, int32_t *__restrict__ counts) {
   const size_t total = (size_t)Ktot * D;
+  wait_prior_grid();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
     const int k = (int)(i / D);
     const long long n = cnt[k];
@@ -866,7 +898,7 @@ static void launch_staged(const UpdateArgs &a, const int32_t *perm, const int32_
   }
   const long long nchunks = ((long long)Ntot + R - 1) / R;
   const int grid = (int)((nchunks + kSegWarps - 1) / kSegWarps);
-  segsum_staged_kernel<T, NACC, MODE><<<grid, kSegWarps * 32, smem, s>>>((const T *)a.X, a.D, perm, skeys, Ntot,
+  launch_chained(segsum_staged_kernel<T, NACC, MODE>, dim3(grid), dim3(kSegWarps * 32), smem, s, (const T *)a.X, a.D, perm, skeys, Ntot,
                                                                         Ktot, R, a.C, a.acc, parts, off);
 }
 
@@ -884,7 +916,7 @@ static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_
     if (aligned && (D * (int)sizeof(T)) % 16 == 0 && (W == 8 || W == 16 || W == 32)) {
       const int ggrid = (int)((nworkers * W + 255) / 256);
 #define FK_GATHER(WW)                                                                                 \
-  return (void)segsum_gather_kernel<T, WW, MODE><<<ggrid, 256, 0, s>>>(X, D, perm, skeys, Ntot, Ktot, R, a.C, \
+  return (void)launch_chained(segsum_gather_kernel<T, WW, MODE>, dim3(ggrid), dim3(256), 0, s, X, D, perm, skeys, Ntot, Ktot, R, a.C, \
                                                                        a.acc, parts, off)
       if (W == 8) FK_GATHER(8);
       if (W == 16) FK_GATHER(16);
@@ -902,7 +934,7 @@ static void launch_segsum(const UpdateArgs &a, const int32_t *perm, const int32_
   const int grid = (int)((nchunks + 7) / 8);
   const bool contig_ok = D % 32 == 0 && aligned;
 #define FK_SEG(NA, CG) \
-  segsum_kernel<T, NA, CG, MODE><<<grid, 256, 0, s>>>(X, D, perm, skeys, Ntot, Ktot, R, a.C, a.acc, parts, off)
+  launch_chained(segsum_kernel<T, NA, CG, MODE>, dim3(grid), dim3(256), 0, s, X, D, perm, skeys, Ntot, Ktot, R, a.C, a.acc, parts, off)
   if (contig_ok && nacc_c == 1) FK_SEG(1, true);
   else if (contig_ok && nacc_c == 2) FK_SEG(2, true);
   else if (contig_ok && nacc_c == 4) FK_SEG(4, true);
@@ -945,19 +977,19 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
   for (int pass = 0; pass < sp.npass; ++pass) {
     const int nbins = 1 << sp.bits[pass];
     if (pass == 0)
-      radix_hist_kernel<true><<<sp.T, kSortThreads, 0, s>>>(kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
+      launch_chained(radix_hist_kernel<true>, dim3(sp.T), dim3(kSortThreads), 0, s, kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
                                                             sp.T, w.H, ctl.status);
     else
-      radix_hist_kernel<false><<<sp.T, kSortThreads, 0, s>>>(kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
+      launch_chained(radix_hist_kernel<false>, dim3(sp.T), dim3(kSortThreads), 0, s, kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
                                                              sp.T, w.H, ctl.status);
-    scan_rows_kernel<<<(nbins + 7) / 8, 256, 0, s>>>(w.H, sp.T, nbins, w.totals);
+    launch_chained(scan_rows_kernel, dim3((nbins + 7) / 8), dim3(256), 0, s, w.H, sp.T, nbins, w.totals);
     const size_t shb = scatter_smem_bytes(nbins);
     if (pass == 0)
-      radix_scatter_kernel<true><<<sp.T, kSortThreads, shb, s>>>(kin, vin, kout, vout, N, a.N, a.K, a.B,
+      launch_chained(radix_scatter_kernel<true>, dim3(sp.T), dim3(kSortThreads), shb, s, kin, vin, kout, vout, N, a.N, a.K, a.B,
                                                                  sp.shift[pass], nbins, sp.T, w.H,
                                                                  w.totals, ctl.status);
     else
-      radix_scatter_kernel<false><<<sp.T, kSortThreads, shb, s>>>(kin, vin, kout, vout, N, a.N, a.K, a.B,
+      launch_chained(radix_scatter_kernel<false>, dim3(sp.T), dim3(kSortThreads), shb, s, kin, vin, kout, vout, N, a.N, a.K, a.B,
                                                                   sp.shift[pass], nbins, sp.T, w.H,
                                                                   w.totals, ctl.status);
     nl += 3;
@@ -986,13 +1018,13 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
   const int fgrid = (int)((fwarps + 7) / 8);
   const int hgrid = (int)(Ktot < (long long)num_sms ? Ktot : (long long)num_sms);
   if (a.mode == kMean) {
-    seg_finalize_kernel<kMean><<<fgrid, 256, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
+    launch_chained(seg_finalize_kernel<kMean>, dim3(fgrid), dim3(256), 0, s, w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
                                                      nullptr, nullptr);
-    seg_finalize_hot_kernel<kMean><<<hgrid, 1024, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, a.C, nullptr);
+    launch_chained(seg_finalize_hot_kernel<kMean>, dim3(hgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts, a.C, nullptr);
   } else {
-    seg_finalize_kernel<kAccumulate><<<fgrid, 256, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr,
+    launch_chained(seg_finalize_kernel<kAccumulate>, dim3(fgrid), dim3(256), 0, s, w.off, (int)Ktot, a.D, R, w.parts, nullptr,
                                                            nullptr, a.acc, a.cnt);
-    seg_finalize_hot_kernel<kAccumulate><<<hgrid, 1024, 0, s>>>(w.off, (int)Ktot, a.D, R, w.parts, nullptr, a.acc);
+    launch_chained(seg_finalize_hot_kernel<kAccumulate>, dim3(hgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts, nullptr, a.acc);
   }
   nl += 3;
   count_launches(nl);
@@ -1005,7 +1037,7 @@ cudaError_t launch_divide_accumulated(double *acc, long long *cnt, int Ktot, int
   long long g = (long long)((total + 255) / 256);
   if (g > 8192) g = 8192;
   if (g < 1) g = 1;
-  divide_acc_kernel<<<(int)g, 256, 0, s>>>(acc, cnt, Ktot, D, C, counts);
+  launch_chained(divide_acc_kernel, dim3((int)g), dim3(256), 0, s, acc, cnt, Ktot, D, C, counts);
   count_launches(1);
   return cudaGetLastError();
 }
