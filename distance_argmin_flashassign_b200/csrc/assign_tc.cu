@@ -71,17 +71,23 @@ constexpr int kBiasBytes = kHalfN * kBiasRow;  // bias terms of a half tile, 4 K
 constexpr int kOnesBytes = 256;             // the tf32 A operand of the bias step
 constexpr int kAcc = 2;                     // accumulators
 constexpr int kEpiWarps = 8;                // column half x lane quarter
-constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
-constexpr int kThreads = 32 * (kEpiWarps + 2);
+// warp 8 loads X, warp 9 issues the MMAs, warp 10 loads the centroid tiles
+constexpr int kProducerWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1, kTileWarp = kEpiWarps + 2;
+constexpr int kThreads = 32 * (kEpiWarps + 3);
 constexpr uint32_t kTmemCols = 512;         // two 256-column fp32 accumulators
 constexpr uint16_t kBothCtas = 0x3;
 static_assert(kAcc * kTileN <= (int)kTmemCols, "accumulators exceed TMEM");
 static_assert(kTileN == kCentroidPad, "the bias is padded to whole tiles");
 
-template <int KB> struct TcCfg {
-  static constexpr int XBUF = 2;                   // X double buffer (next unit prefetch)
+// Shared-memory plan.  With many tiles per unit the X tile of the next unit
+// has several tiles' time to load, and the ring holds as many tile slots as
+// fit.  With at most two tiles per unit (small K, e.g. a batch of small
+// problems) a unit's MMAs last less than one X load takes, so the deep-X
+// plan (DX) keeps several units of X in flight and only two tile slots.
+template <int KB, bool DX> struct TcCfg {
+  static constexpr int XBUF = DX ? (KB == 1 ? 8 : 4) : 2;  // X buffers (units in flight)
   static constexpr int SLOT = KB * kStageBytes + kBiasBytes;  // one tile's centroids and bias terms
-  static constexpr int NSLOT = KB == 1 ? 9 : 4;    // tile slots in the ring
+  static constexpr int NSLOT = DX ? (KB == 1 ? 4 : 2) : (KB == 1 ? 9 : 4);  // tile slots in the ring
   static constexpr int X_BYTES = XBUF * KB * kXBytes;
   static constexpr int C_BYTES = NSLOT * SLOT;
   static constexpr int XCHG_BYTES = kRows * 16;    // one float4 per row
@@ -192,17 +198,23 @@ __device__ __forceinline__ void fold_chunk(Best &bs, const uint32_t (&v)[32], in
   }
 }
 
-template <int KB>
+template <int KB, bool DX>
 __global__ void __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
                      const __grid_constant__ CUtensorMap bmap, const TcParams p) {
-  using Cfg = TcCfg<KB>;
+  using Cfg = TcCfg<KB, DX>;
   constexpr int NST = Cfg::NSLOT, XBUF = Cfg::XBUF;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
 
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  // The pair's units: a contiguous range, so that consecutive units mostly
+  // belong to the same problem (a batch of problems reuses its centroid
+  // tiles from one unit to the next, see the producer).
+  const int upp = (p.total_units + npairs - 1) / npairs;
+  const int u_begin = pair * upp;
+  const int u_end = u_begin + upp < p.total_units ? u_begin + upp : p.total_units;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
   // Both CTAs of a pair see the same layout (same kernel, same dynamic size),
@@ -274,10 +286,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer ----
-      uint32_t xb = 0, xph = 0, st = 0, sph = 0;
-      bool ok = true, issued = false, waited = false;
-      for (int u = pair; ok && u < p.total_units; u += npairs) {
+      // ------------------------------------------------- X producer -----
+      // X streams up to XBUF units ahead of the MMAs, independently of the
+      // centroid tiles (a unit of one or two tiles is over before one X
+      // tile has loaded)
+      uint32_t xb = 0, xph = 0;
+      bool ok = true, issued = false;
+      for (int u = u_begin; ok && u < u_end; ++u) {
         const int b = u / p.upb, r0 = (u % p.upb) * kRowsUnit + (int)rank * kRows;
         if (!(ok = mbar_wait(xempty(xb), xph ^ 1u, abort_flag, p.ctl))) break;
         if (leader) mbar_arrive_expect_tx(xfull(xb), 2 * KB * kXBytes);
@@ -286,26 +301,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d_pair(sX + (xb * KB + kb) * kXBytes, &xmap, xbar, kb * kBlkK, r0, b);
         issued = true;
         if (++xb == XBUF) { xb = 0; xph ^= 1u; }
-        if (!waited) {
-          // The kernel may be launched before the one that prepared the
-          // centroids and the bias has finished (programmatic stream
-          // serialization): X is input only and loads at once, the centroid
-          // tiles wait until that kernel's writes are visible.
-          asm volatile("griddepcontrol.wait;" ::: "memory");
-          waited = true;
-        }
-        for (int j = 0; ok && j < p.ntiles; ++j) {
-          if (!(ok = mbar_wait(empty(st), sph ^ 1u, abort_flag, p.ctl))) break;
-          if (leader) mbar_arrive_expect_tx(full(st), 2 * (KB * kStageBytes + kBiasBytes));
-          const uint32_t fbar = map_to_cta(full(st), 0);
-          const int c0 = j * kTileN + (int)rank * kHalfN;
-          for (int kb = 0; kb < KB; ++kb) tma_load_3d_pair(slot_c(st, kb), &cmap, fbar, kb * kBlkK, c0, b);
-          tma_load_3d_pair(slot_bias(st), &bmap, fbar, 0, c0, b);
-          if (++st == NST) { st = 0; sph ^= 1u; }
-        }
       }
       // After an abort, give copies already issued time to land in this CTA's
       // shared memory before it can exit (their barrier may be in the peer).
+      if (!ok && issued) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 50000ull) {
+        }
+      }
+    }
+  } else if (warp == kTileWarp) {
+    if (lane == 0) {
+      // ---------------------------------------------- tile producer -----
+      // The kernel may be launched before the one that prepared the
+      // centroids and the bias has finished (programmatic stream
+      // serialization): the centroid tiles wait until that kernel's writes
+      // are visible.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      uint32_t st = 0, sph = 0;
+      bool ok = true, issued = false;
+      // (problem, tile) + 1 held by each slot, 0 when not known: both CTAs of
+      // the pair track it alike, so both skip or both load
+      int held[NST];
+      for (int i = 0; i < NST; ++i) held[i] = 0;
+      for (int u = u_begin; ok && u < u_end; ++u) {
+        const int b = u / p.upb;
+        for (int j = 0; ok && j < p.ntiles; ++j) {
+          if (!(ok = mbar_wait(empty(st), sph ^ 1u, abort_flag, p.ctl))) break;
+          const int tag = b * p.ntiles + j + 1;
+          if (held[st] == tag) {
+            // the slot already holds this tile (same problem, one or two
+            // tiles per unit): hand it over again without copying
+            if (leader) mbar_arrive(full(st));
+          } else {
+            if (leader) mbar_arrive_expect_tx(full(st), 2 * (KB * kStageBytes + kBiasBytes));
+            const uint32_t fbar = map_to_cta(full(st), 0);
+            const int c0 = j * kTileN + (int)rank * kHalfN;
+            for (int kb = 0; kb < KB; ++kb) tma_load_3d_pair(slot_c(st, kb), &cmap, fbar, kb * kBlkK, c0, b);
+            tma_load_3d_pair(slot_bias(st), &bmap, fbar, 0, c0, b);
+            held[st] = tag;
+            issued = true;
+          }
+          if (++st == NST) { st = 0; sph ^= 1u; }
+        }
+      }
       if (!ok && issued) {
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 50000ull) {
@@ -319,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t ones_desc = desc_ones(smem_u32(ones));
       int t = 0;  // tile counter: accumulator t % 2, its (t / 2)-th use
       bool ok = true;
-      for (int u = pair; ok && u < p.total_units; u += npairs) {
+      for (int u = u_begin; ok && u < u_end; ++u) {
         if (!(ok = mbar_wait(xfull(xb), xph, abort_flag, p.ctl))) break;
         const uint32_t xa = sX + xb * KB * kXBytes;
         for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
@@ -371,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t xb = 0, xc = 0;
     int t = 0;  // the pair's tile counter
     bool ok = true;
-    for (int u = pair; ok && u < p.total_units; u += npairs, xc ^= 1u) {
+    for (int u = u_begin; ok && u < u_end; ++u, xc ^= 1u) {
       const int b = u / p.upb;
       const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
       Best bs;
@@ -420,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // merge the two column halves of each point: half 1 hands over its
       // candidate and |x|^2, half 0 merges and writes
       if (h == 1) {
-        if (u != pair && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
+        if (u != u_begin && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
         float xn = 0.f;
         if (p.mindist) {
           // |x|^2 from the swizzled X tile: every MMA of this unit is done
@@ -536,7 +575,7 @@ bool tc_aligned(const void *X, const void *C) {
   return ((uintptr_t)X % 16 == 0) && ((uintptr_t)C % 16 == 0);
 }
 
-template <int KB>
+template <int KB, bool DX>
 static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, TcParams p,
                              int num_sms, cudaStream_t s) {
   static int configured[64] = {};
@@ -545,12 +584,12 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   cudaGetDevice(&dev);
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int want = TcCfg<KB>::USED + 1024;
+  const int want = TcCfg<KB, DX>::USED + 1024;
   const int dyn = want < optin ? want : optin;
   {
     std::lock_guard<std::mutex> g(mu);
     if (dev < 64 && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB, DX>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
       if (e != cudaSuccess) return e;
       configured[dev] = 1;
     }
@@ -574,7 +613,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB>, xm, cm, bm, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB, DX>, xm, cm, bm, p);
   count_launches(1);
   return e;
 }
@@ -604,8 +643,9 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   if (p.total_units == 0) return cudaSuccess;
   if (Kpad < p.ntiles * kTileN) return cudaErrorInvalidValue;  // the bias must cover every tile
   const int KB = (D + kBlkK - 1) / kBlkK;
-  if (KB == 1) return launch_kb<1>(xm, cm, bm, p, num_sms, s);
-  return launch_kb<2>(xm, cm, bm, p, num_sms, s);
+  const bool deep_x = p.ntiles <= 2;
+  if (KB == 1) return deep_x ? launch_kb<1, true>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false>(xm, cm, bm, p, num_sms, s);
+  return deep_x ? launch_kb<2, true>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false>(xm, cm, bm, p, num_sms, s);
 }
 
 }  // namespace fk
