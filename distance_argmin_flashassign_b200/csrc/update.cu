@@ -7,7 +7,7 @@
 //   1. stable LSD radix sort of the cluster ids (11-bit digits, one pass for
 //      up to 2,048 clusters, two for up to 2^22): per-tile digit histograms,
 //      a per-digit scan over tiles, and a scatter whose within-tile ranks come
-//      from warp-level match_any -- the sorted point ids are the inverse map
+//      from warp ballots -- the sorted point ids are the inverse map
 //      (cluster -> its points);
 //   2. segmented sums: the sorted order is cut into equal chunks of R
 //      positions, one warp per chunk, so a hot cluster (Zipf skew) is spread
@@ -182,6 +182,16 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   uint16_t *wcnt = reinterpret_cast<uint16_t *>(vals_s + kSortTile);  // [8][nbins + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   wait_prior_grid();
+  // the warp's 512 consecutive keys and values are loaded first, so that
+  // their latency overlaps the digit-base reads below
+  int keyr[kSortItems], valr[kSortItems], locr[kSortItems];
+  const int base = blockIdx.x * kSortTile + warp * (kSortItems * 32);
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it) {
+    const int pos = base + it * 32 + lane;
+    keyr[it] = pos < Ntot ? keys_in[pos] : 0;
+    valr[it] = pos < Ntot ? (FIRST ? pos : vals_in[pos]) : 0;
+  }
 
   // digit base of this tile = exclusive scan of digit totals + tile prefix
   const int per = (nbins + kSortThreads - 1) / kSortThreads;
@@ -209,31 +219,32 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     }
   }
 
-  // stable ranks within each warp's 512 consecutive keys
-  int keyr[kSortItems], valr[kSortItems], locr[kSortItems];
-  const int base = blockIdx.x * kSortTile + warp * (kSortItems * 32);
+  // stable ranks within each warp's 512 consecutive keys.  The lanes that
+  // hold the same digit are found with one ballot per digit bit: a fixed
+  // cost, where match.any's grows with the number of distinct digits (up to
+  // 32 here, with 1024 or more bins).
   const unsigned lt_mask = (1u << lane) - 1u;
+  const int dbits = __ffs(nbins) - 1;
   uint16_t *mycnt = wcnt + warp * stride;
-  // all of the warp's keys and values are loaded before the ranking starts
-#pragma unroll
-  for (int it = 0; it < kSortItems; ++it) {
-    const int pos = base + it * 32 + lane;
-    keyr[it] = pos < Ntot ? keys_in[pos] : 0;
-    valr[it] = pos < Ntot ? (FIRST ? pos : vals_in[pos]) : 0;
-  }
   bool bad = false;
 #pragma unroll
   for (int it = 0; it < kSortItems; ++it) {
     const int pos = base + it * 32 + lane;
-    int d = nbins;
-    if (pos < Ntot) {
+    const bool valid = pos < Ntot;
+    int d = 0;
+    if (valid) {
       if (FIRST) keyr[it] = key_of_label(keyr[it], pos, N, K, B, bad);
       d = (keyr[it] >> shift) & (nbins - 1);
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, d);
-    const int c = mycnt[d];
+    unsigned peers = __ballot_sync(0xffffffffu, valid);
+    for (int b = 0; b < dbits; ++b) {
+      const bool bit = (d >> b) & 1;
+      const unsigned m = __ballot_sync(0xffffffffu, bit);
+      peers &= bit ? m : ~m;
+    }
+    const int c = valid ? mycnt[d] : 0;
     __syncwarp();
-    if (lane == __ffs(peers) - 1) mycnt[d] = (uint16_t)(c + __popc(peers));
+    if (valid && lane == __ffs(peers) - 1) mycnt[d] = (uint16_t)(c + __popc(peers));
     __syncwarp();
     locr[it] = c + __popc(peers & lt_mask);
   }
