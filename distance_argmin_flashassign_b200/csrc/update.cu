@@ -163,8 +163,13 @@ __global__ void __launch_bounds__(256) scan_rows_kernel(int *__restrict__ H, int
   if (lane == 0) totals[w] = carry;
 }
 
+// ints of the region that holds the warps' digit masks while keys are
+// ranked, then the tile's keys and values in sorted order
+static __host__ __device__ int scatter_xbuf_ints(int nbins) {
+  return 2 * kSortTile > kSortWarps * nbins ? 2 * kSortTile : kSortWarps * nbins;
+}
 static size_t scatter_smem_bytes(int nbins) {
-  return (size_t)(2 * nbins + 8 + 2 * kSortTile) * 4 + (size_t)kSortWarps * (nbins + 1) * 2;
+  return (size_t)(2 * nbins + kSortWarps + scatter_xbuf_ints(nbins)) * 4 + (size_t)kSortWarps * (nbins + 1) * 4;
 }
 
 template <bool FIRST>
@@ -176,10 +181,11 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   const int stride = nbins + 1;
   int *dbase = sh;                                                   // [nbins]
   int *tstart = sh + nbins;                                          // [nbins]
-  int *wsum = sh + 2 * nbins;                                        // [8]
-  int *keys_s = sh + 2 * nbins + 8;                                  // [kSortTile]
+  int *wsum = sh + 2 * nbins;                                        // [kSortWarps]
+  int *keys_s = sh + 2 * nbins + kSortWarps;                         // [kSortTile]
   int *vals_s = keys_s + kSortTile;                                  // [kSortTile]
-  uint16_t *wcnt = reinterpret_cast<uint16_t *>(vals_s + kSortTile);  // [8][nbins + 1]
+  unsigned *wmask = reinterpret_cast<unsigned *>(keys_s);            // [kSortWarps][nbins], same place
+  int *wcnt = keys_s + scatter_xbuf_ints(nbins);                     // [kSortWarps][nbins + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   wait_prior_grid();
   // the warp's 512 consecutive keys and values are loaded first, so that
@@ -193,13 +199,21 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     valr[it] = pos < Ntot ? (FIRST ? pos : vals_in[pos]) : 0;
   }
 
-  // digit base of this tile = exclusive scan of digit totals + tile prefix
+  // digit base of this tile = exclusive scan of digit totals + tile prefix;
+  // both reads of a thread's digits are issued before either is used
+  constexpr int kPer = kMaxBins / kSortThreads;  // digits per thread, at most
   const int per = (nbins + kSortThreads - 1) / kSortThreads;
-  int s = 0;
-  for (int i = 0; i < per; ++i) {
+  int tv[kPer], hv[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
     const int d = tid * per + i;
-    if (d < nbins) s += totals[d];
+    const bool ok = i < per && d < nbins;
+    tv[i] = ok ? totals[d] : 0;
+    hv[i] = ok ? H[(size_t)d * T + blockIdx.x] : 0;
   }
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) s += tv[i];
   int incl = s;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -208,24 +222,29 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   }
   if (lane == 31) wsum[warp] = incl;
   for (int i = tid; i < kSortWarps * stride; i += kSortThreads) wcnt[i] = 0;
+  for (int i = tid; i < kSortWarps * nbins; i += kSortThreads) wmask[i] = 0u;
   __syncthreads();
   int run = incl - s;
   for (int w = 0; w < warp; ++w) run += wsum[w];
-  for (int i = 0; i < per; ++i) {
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
     const int d = tid * per + i;
-    if (d < nbins) {
-      dbase[d] = run + H[(size_t)d * T + blockIdx.x];
-      run += totals[d];
-    }
+    if (i < per && d < nbins) dbase[d] = run + hv[i];
+    run += tv[i];
   }
 
-  // stable ranks within each warp's 512 consecutive keys.  The lanes that
-  // hold the same digit are found with one ballot per digit bit: a fixed
-  // cost, where match.any's grows with the number of distinct digits (up to
-  // 32 here, with 1024 or more bins).
+  // stable ranks within each warp's consecutive keys.  The lanes that hold
+  // the same digit find each other through shared memory: each sets its bit
+  // in the warp's mask word of its digit and reads the word back (on this
+  // GPU much cheaper than a ballot per digit bit or match.any, whose cost
+  // grows with the number of distinct digits).  The lowest of them clears
+  // the word and adds the group's size to the warp's count of that digit;
+  // the count before the add, broadcast after all of the warp's keys are
+  // counted, is where the group starts.
   const unsigned lt_mask = (1u << lane) - 1u;
-  const int dbits = __ffs(nbins) - 1;
-  uint16_t *mycnt = wcnt + warp * stride;
+  int *mycnt = wcnt + warp * stride;
+  unsigned *mymask = wmask + warp * nbins;
+  unsigned peer[kSortItems];
   bool bad = false;
 #pragma unroll
   for (int it = 0; it < kSortItems; ++it) {
@@ -236,24 +255,28 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
       if (FIRST) keyr[it] = key_of_label(keyr[it], pos, N, K, B, bad);
       d = (keyr[it] >> shift) & (nbins - 1);
     }
-    unsigned peers = __ballot_sync(0xffffffffu, valid);
-    for (int b = 0; b < dbits; ++b) {
-      const bool bit = (d >> b) & 1;
-      const unsigned m = __ballot_sync(0xffffffffu, bit);
-      peers &= bit ? m : ~m;
+    if (valid) atomicOr(mymask + d, 1u << lane);
+    __syncwarp();
+    const unsigned peers = valid ? mymask[d] : 0u;
+    __syncwarp();
+    int c = 0;
+    if (valid && lane == __ffs(peers) - 1) {
+      mymask[d] = 0u;
+      c = atomicAdd(mycnt + d, __popc(peers));
     }
-    const int c = valid ? mycnt[d] : 0;
-    __syncwarp();
-    if (valid && lane == __ffs(peers) - 1) mycnt[d] = (uint16_t)(c + __popc(peers));
-    __syncwarp();
-    locr[it] = c + __popc(peers & lt_mask);
+    __syncwarp();  // the next key's mask and add come after these
+    peer[it] = peers;
+    locr[it] = c;
   }
+#pragma unroll
+  for (int it = 0; it < kSortItems; ++it)
+    locr[it] = __shfl_sync(0xffffffffu, locr[it], (__ffs(peer[it]) - 1) & 31) + __popc(peer[it] & lt_mask);
   if (bad) record_status(status, kStBadLabel);
-  __syncthreads();
+  __syncthreads();  // masks done: the region holds keys and values from here on
   // per digit: exclusive prefix over warps (in place) and the tile's count,
   // then the exclusive scan of the tile's counts over digits: where each
   // digit's run starts in the tile's sorted order
-  int cnt[kMaxBins / kSortThreads];
+  int cnt[kPer];
   int tsum = 0;
   for (int i = 0; i < per; ++i) {
     const int d = tid * per + i;
@@ -261,7 +284,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     if (d < nbins)
       for (int w = 0; w < kSortWarps; ++w) {
         const int t = wcnt[w * stride + d];
-        wcnt[w * stride + d] = (uint16_t)r;
+        wcnt[w * stride + d] = r;
         r += t;
       }
     cnt[i] = r;
