@@ -425,24 +425,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (h == 0 && q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
         const uint32_t ta = t_row + a * kTileN;
         const int col = j * kTileN + h * kHalfN;
-        uint32_t va[32], vb[32];
-        // chunks 0 and 1
+        uint32_t va[32], vb[32], vc[32];
+        // chunks 0 and 1; the loads of chunks 2 and 3 are issued while they
+        // are folded (chunk 3 into chunk 0's registers once it is folded)
         FK_TMEM_LD32(ta, va);
         FK_TMEM_LD32(ta + 32, vb);
         FK_TMEM_WAIT_LD(va);
         FK_TMEM_WAIT_LD(vb);
+        FK_TMEM_LD32(ta + 64, vc);
         fold_chunk(bs, va, col);
+        FK_TMEM_LD32(ta + 96, va);
         fold_chunk(bs, vb, col + 32);
         // chunks 2 and 3: once they are in registers the accumulator is free
-        FK_TMEM_LD32(ta + 64, va);
-        FK_TMEM_LD32(ta + 96, vb);
+        FK_TMEM_WAIT_LD(vc);
         FK_TMEM_WAIT_LD(va);
-        FK_TMEM_WAIT_LD(vb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(a);
-        fold_chunk(bs, va, col + 64);
-        fold_chunk(bs, vb, col + 96);
+        fold_chunk(bs, vc, col + 64);
+        fold_chunk(bs, va, col + 96);
       }
       if (!ok) break;
       // lowest column of the candidate chunk holding the maximum
