@@ -654,6 +654,15 @@ __global__ void __launch_bounds__(kSegWarps * 32) segsum_staged_kernel(
 // random rows at full rate.  The segmentation (which segments are whole,
 // which go to the two partial slots of the chunk) is the one of
 // segsum_kernel, with worker index in place of warp index.
+// 16 bytes of a row of X, read once: not kept in L1 (allocating L1 lines for
+// the gathered rows cost the segment sums 7 % on the embedding workload).
+__device__ __forceinline__ uint4 ld_row16(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
 constexpr int kGatherRows = 8;
 template <typename T, int W, int MODE>
 __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restrict__ X, int D,
@@ -717,7 +726,7 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
     for (int u = 0; u < U; ++u) {
       const int row = __shfl_sync(0xffffffffu, mr, u, W);
       kk[u] = __shfl_sync(0xffffffffu, mk, u, W);
-      v[u] = (b0 + u < p1) ? __ldg(reinterpret_cast<const uint4 *>(X + (size_t)row * D) + lw) : make_uint4(0, 0, 0, 0);
+      v[u] = (b0 + u < p1) ? ld_row16(reinterpret_cast<const uint4 *>(X + (size_t)row * D) + lw) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
