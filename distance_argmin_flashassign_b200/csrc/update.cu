@@ -716,25 +716,35 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
   // every worker of the warp runs the same number of batches (shuffles stay
   // converged); positions past a worker's end are masked
   const int nb = (R + U - 1) / U;
+  // lanes 0 .. U-1 hold the sorted keys and point ids of a batch; those of
+  // the next batch are loaded while this batch's rows are in flight, so a
+  // batch costs one memory round trip, not two
+  int mk_next = 0, mr_next = 0;
+  auto batch_ids = [&](int bt) {
+    const int b0 = p0 + bt * U;
+    const bool in = lw < U && b0 + lw < p1;
+    mk_next = in ? skeys[b0 + lw] : 0;
+    mr_next = in ? perm[b0 + lw] : 0;
+  };
+  batch_ids(0);
   for (int bt = 0; bt < nb; ++bt) {
     const int b0 = p0 + bt * U;
-    const int mk = (lw < U && b0 + lw < p1) ? skeys[b0 + lw] : 0;
-    const int mr = (lw < U && b0 + lw < p1) ? perm[b0 + lw] : 0;
+    const int mk = mk_next, mr = mr_next;
     uint4 v[U];
-    int kk[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int row = __shfl_sync(0xffffffffu, mr, u, W);
-      kk[u] = __shfl_sync(0xffffffffu, mk, u, W);
       v[u] = (b0 + u < p1) ? ld_row16(reinterpret_cast<const uint4 *>(X + (size_t)row * D) + lw) : make_uint4(0, 0, 0, 0);
     }
+    if (bt + 1 < nb) batch_ids(bt + 1);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+      const int ku = __shfl_sync(0xffffffffu, mk, u, W);
       if (b0 + u < p1) {
-        if (kk[u] != cur) {
+        if (ku != cur) {
           flush(cur, s, b0 + u);
-          for (int q = cur + 1 + lw; q <= kk[u]; q += W) off[q] = b0 + u;
-          cur = kk[u];
+          for (int q = cur + 1 + lw; q <= ku; q += W) off[q] = b0 + u;
+          cur = ku;
           s = b0 + u;
 #pragma unroll
           for (int i = 0; i < EPL; ++i) a[i] = 0.f;
