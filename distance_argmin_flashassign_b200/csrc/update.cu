@@ -698,6 +698,17 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
   const int p1 = (Ntot - p0) < R ? Ntot : p0 + R;
   int cur = 0, s = p0;
   bool split_start = false, split_end = false;
+  // lanes 0 .. U-1 hold the sorted keys and point ids of a batch; those of
+  // the next batch are loaded while this batch's rows are in flight, so a
+  // batch costs one memory round trip, not two
+  int mk_next = 0, mr_next = 0;
+  auto batch_ids = [&](int bt) {
+    const int b0 = p0 + bt * U;
+    const bool in = lw < U && b0 + lw < p1;
+    mk_next = in ? skeys[b0 + lw] : 0;
+    mr_next = in ? perm[b0 + lw] : 0;
+  };
+  batch_ids(0);  // in flight together with the chunk-boundary keys below
   if (live) {
     const int kfirst = skeys[p0];
     const int kprev = p0 > 0 ? skeys[p0 - 1] : -1;
@@ -732,17 +743,6 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
   // every worker of the warp runs the same number of batches (shuffles stay
   // converged); positions past a worker's end are masked
   const int nb = (R + U - 1) / U;
-  // lanes 0 .. U-1 hold the sorted keys and point ids of a batch; those of
-  // the next batch are loaded while this batch's rows are in flight, so a
-  // batch costs one memory round trip, not two
-  int mk_next = 0, mr_next = 0;
-  auto batch_ids = [&](int bt) {
-    const int b0 = p0 + bt * U;
-    const bool in = lw < U && b0 + lw < p1;
-    mk_next = in ? skeys[b0 + lw] : 0;
-    mr_next = in ? perm[b0 + lw] : 0;
-  };
-  batch_ids(0);
   for (int bt = 0; bt < nb; ++bt) {
     const int b0 = p0 + bt * U;
     const int mk = mk_next, mr = mr_next;
@@ -789,119 +789,103 @@ __global__ void __launch_bounds__(256, 3) segsum_gather_kernel(const T *__restri
   }
 }
 
-// One warp per cluster (grid-stride): the count, then, for a segment that
-// crosses chunk borders but has at most kHotParts partial rows, the sum of
-// those rows in chunk order (two interleaved running sums, added at the end:
-// a fixed order), divided by the count.  Segments inside one chunk were
-// written by their worker; segments with more partial rows (the hot clusters
-// of a skewed distribution) are left to seg_finalize_hot_kernel.
+// Per cluster: the count and, for a segment that crosses chunk borders, the
+// sum of its partial rows in a fixed order, divided by the count (segments
+// inside one chunk were written by their segment-sum worker).  Block b of G
+// owns the clusters b, b + G, b + 2G, ... (hot clusters of a skewed
+// distribution are usually consecutive ids, so they land in different
+// blocks) and takes them 1024 at a time.  Warp w handles the window's
+// clusters w, w + 32, ...: a segment with at most kHotParts partial rows it
+// sums itself (lanes over dimensions, rows in chunk order); longer ones are
+// listed in shared memory and summed after the window by all 32 warps: warp
+// w sums the partial rows w, w + 32, ..., then thread d adds the 32 warp sums
+// of dimension d in warp order.
 constexpr int kHotParts = 16;
 template <int MODE>
-__global__ void __launch_bounds__(256) seg_finalize_kernel(const int *__restrict__ off, int Ktot, int D, int R,
-                                                           const float *__restrict__ parts,
-                                                           float *__restrict__ C, int32_t *__restrict__ counts,
-                                                           double *__restrict__ acc, long long *__restrict__ cnt) {
-  const int lane = threadIdx.x & 31;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  wait_prior_grid();
-  for (long long k = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; k < Ktot; k += nw) {
-    const int s = off[k], e = off[k + 1], n = e - s;
-    if (lane == 0) {
-      if (MODE == kMean) {
-        if (counts) counts[k] = n;
-      } else {
-        cnt[k] += n;
-      }
-    }
-    if (n == 0) continue;
-    const int q0 = s / R, q1 = (e - 1) / R;
-    if (q0 == q1) continue;  // segment inside one chunk: already written
-    const int np = q1 - q0 + 1;
-    if (np > kHotParts) continue;
-    const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
-    auto part_row = [&](int i) { return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D; };
-    // 4 dimensions per lane per pass; every partial row's loads are
-    // independent of the running sums, so they are all in flight together
-    for (int d0 = 0; d0 < D; d0 += 128) {
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i = 0; i < np; ++i) {
-        const float *row = part_row(i) + d0;
-        float v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = d0 + lane + 32 * j < D ? row[lane + 32 * j] : 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) t[j] += v[j];
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int d = d0 + lane + 32 * j;
-        if (d >= D) continue;
-        if (MODE == kMean) C[(size_t)k * D + d] = t[j] / (float)n;
-        else acc[(size_t)k * D + d] += (double)t[j];
-      }
-    }
-  }
-}
-
-// Segments with more than kHotParts partial rows.  Block b owns the clusters
-// b, b + G, b + 2G, ... (G blocks; hot clusters of a skewed distribution are
-// usually consecutive ids, so they land in different blocks).  It looks at
-// 1024 of them at once (one per thread), lists the hot ones in shared
-// memory, then gives each of them all of its 32 warps: warp w sums
-// the partial rows w, w + 32, ... (lanes over dimensions), then thread d adds
-// the 32 warp sums of dimension d in warp order: a fixed order.
-template <int MODE>
-__global__ void __launch_bounds__(1024) seg_finalize_hot_kernel(const int *__restrict__ off, int Ktot, int D, int R,
-                                                                const float *__restrict__ parts,
-                                                                float *__restrict__ C, double *__restrict__ acc) {
+__global__ void __launch_bounds__(1024) seg_finalize_kernel(const int *__restrict__ off, int Ktot, int D, int R,
+                                                            const float *__restrict__ parts,
+                                                            float *__restrict__ C, int32_t *__restrict__ counts,
+                                                            double *__restrict__ acc, long long *__restrict__ cnt) {
   __shared__ float red[32][129];
   __shared__ int hot[1024];
   __shared__ int nhot;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   wait_prior_grid();
   const long long G = gridDim.x;
+  auto part_row = [&](int s, int q0, int i) {
+    const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
+    return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D;
+  };
+  auto emit = [&](int k, int d, float sum, int n) {
+    const size_t o = (size_t)k * D + d;
+    if (MODE == kMean) C[o] = sum / (float)n;
+    else acc[o] += (double)sum;
+  };
   for (long long i0 = 0; blockIdx.x + G * i0 < Ktot; i0 += 1024) {
     if (threadIdx.x == 0) nhot = 0;
     __syncthreads();
-    {
-      const long long kl = blockIdx.x + G * (i0 + threadIdx.x);
+    for (int j = w; j < 1024; j += 32) {
+      const long long kl = blockIdx.x + G * (i0 + j);
+      if (kl >= Ktot) break;
       const int k = (int)kl;
-      if (kl < Ktot) {
-        const int s = off[k], e = off[k + 1];
-        if (e > s && (e - 1) / R - s / R + 1 > kHotParts) hot[atomicAdd(&nhot, 1)] = k;
+      const int s = off[k], e = off[k + 1], n = e - s;
+      if (lane == 0) {
+        if (MODE == kMean) {
+          if (counts) counts[k] = n;
+        } else {
+          cnt[k] += n;
+        }
+      }
+      if (n == 0) continue;
+      const int q0 = s / R, q1 = (e - 1) / R;
+      if (q0 == q1) continue;  // segment inside one chunk: already written
+      const int np = q1 - q0 + 1;
+      if (np > kHotParts) {
+        if (lane == 0) hot[atomicAdd(&nhot, 1)] = k;
+        continue;
+      }
+      // 4 dimensions per lane per pass; every partial row's loads are
+      // independent of the running sums, so they are all in flight together
+      for (int d0 = 0; d0 < D; d0 += 128) {
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = 0; i < np; ++i) {
+          const float *row = part_row(s, q0, i) + d0;
+          float v[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) v[jj] = d0 + lane + 32 * jj < D ? row[lane + 32 * jj] : 0.f;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) t[jj] += v[jj];
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          if (d0 + lane + 32 * jj < D) emit(k, d0 + lane + 32 * jj, t[jj], n);
       }
     }
     __syncthreads();
     const int nh = nhot;
     for (int h = 0; h < nh; ++h) {
-    const int k = hot[h];
-    const int s = off[k], e = off[k + 1], n = e - s;
-    const int q0 = s / R, q1 = (e - 1) / R;
-    const int np = q1 - q0 + 1;
-    const size_t first = (size_t)q0 * 2 + (s == q0 * R ? 0 : 1);
-    auto part_row = [&](int i) { return parts + (i == 0 ? first : (size_t)(q0 + i) * 2) * D; };
-    for (int d0 = 0; d0 < D; d0 += 128) {
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i = w; i < np; i += 32) {
-        const float *row = part_row(i) + d0;
+      const int k = hot[h];
+      const int s = off[k], e = off[k + 1], n = e - s;
+      const int q0 = s / R, np = (e - 1) / R - q0 + 1;
+      for (int d0 = 0; d0 < D; d0 += 128) {
+        float t[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = w; i < np; i += 32) {
+          const float *row = part_row(s, q0, i) + d0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (d0 + lane + 32 * j < D) t[j] += row[lane + 32 * j];
-      }
+          for (int jj = 0; jj < 4; ++jj)
+            if (d0 + lane + 32 * jj < D) t[jj] += row[lane + 32 * jj];
+        }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) red[w][lane + 32 * j] = t[j];
-      __syncthreads();
-      if (threadIdx.x < 128 && d0 + threadIdx.x < D) {
-        float tot = 0.f;
-        for (int ww = 0; ww < 32; ++ww) tot += red[ww][threadIdx.x];
-        const size_t o = (size_t)k * D + d0 + threadIdx.x;
-        if (MODE == kMean) C[o] = tot / (float)n;
-        else acc[o] += (double)tot;
+        for (int jj = 0; jj < 4; ++jj) red[w][lane + 32 * jj] = t[jj];
+        __syncthreads();
+        if (threadIdx.x < 128 && d0 + threadIdx.x < D) {
+          float tot = 0.f;
+          for (int ww = 0; ww < 32; ++ww) tot += red[ww][threadIdx.x];
+          emit(k, d0 + threadIdx.x, tot, n);
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
-    }
-    __syncthreads();  // the list is rebuilt for the next window
   }
 }
 
@@ -1083,19 +1067,16 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
       a.mode == kMean ? launch_segsum<__nv_bfloat16, kMean>(a, perm, skeys, N, KT, R, w.parts, w.off, s)
                       : launch_segsum<__nv_bfloat16, kAccumulate>(a, perm, skeys, N, KT, R, w.parts, w.off, s);
   }
-  const long long fwarps = Ktot < (long long)num_sms * 64 ? Ktot : (long long)num_sms * 64;
-  const int fgrid = (int)((fwarps + 7) / 8);
-  const int hgrid = (int)(Ktot < (long long)num_sms ? Ktot : (long long)num_sms);
-  if (a.mode == kMean) {
-    launch_chained(seg_finalize_kernel<kMean>, dim3(fgrid), dim3(256), 0, s, w.off, (int)Ktot, a.D, R, w.parts, a.C, a.counts,
-                                                     nullptr, nullptr);
-    launch_chained(seg_finalize_hot_kernel<kMean>, dim3(hgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts, a.C, nullptr);
-  } else {
-    launch_chained(seg_finalize_kernel<kAccumulate>, dim3(fgrid), dim3(256), 0, s, w.off, (int)Ktot, a.D, R, w.parts, nullptr,
-                                                           nullptr, a.acc, a.cnt);
-    launch_chained(seg_finalize_hot_kernel<kAccumulate>, dim3(hgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts, nullptr, a.acc);
-  }
-  nl += 3;
+  // one block of 32 warps per 32 clusters, at most one per SM
+  long long fgrid = (Ktot + 31) / 32;
+  if (fgrid > num_sms) fgrid = num_sms;
+  if (a.mode == kMean)
+    launch_chained(seg_finalize_kernel<kMean>, dim3((int)fgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts, a.C,
+                   a.counts, nullptr, nullptr);
+  else
+    launch_chained(seg_finalize_kernel<kAccumulate>, dim3((int)fgrid), dim3(1024), 0, s, w.off, (int)Ktot, a.D, R, w.parts,
+                   nullptr, nullptr, a.acc, a.cnt);
+  nl += 2;
   count_launches(nl);
   return cudaGetLastError();
 }
