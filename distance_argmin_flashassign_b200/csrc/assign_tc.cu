@@ -254,11 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < XBUF; ++x) {
       mbar_init(xfull(x), 1);
-      mbar_init(xempty(x), kEpiWarps);  // this CTA's epilogue warps, after the unit
+      mbar_init(xempty(x), p.ntiles == 1 ? kEpiWarps / 2 : kEpiWarps);  // this CTA's warps of the unit, after it
     }
+    // With one tile per unit each unit is read by one warp of each lane
+    // quarter (see the epilogue), else by all epilogue warps.
+    const int readers = p.ntiles == 1 ? kEpiWarps / 2 : kEpiWarps;
     for (int a = 0; a < kAcc; ++a) {
-      mbar_init(accfull(a), 1);               // the MMA commit
-      mbar_init(accempty(a), 2 * kEpiWarps);  // every epilogue warp of both CTAs
+      mbar_init(accfull(a), 1);             // the MMA commit
+      mbar_init(accempty(a), 2 * readers);  // those epilogue warps of both CTAs
     }
     mbar_init(xchg_full, kEpiWarps / 2);   // the column-half-1 warps
     mbar_init(xchg_empty, kEpiWarps / 2);  // the column-half-0 warps
@@ -393,60 +396,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ epilogue ----
     const int h = warp >> 2, q = warp & 3;  // column half, lane quarter
     const int r = q * 32 + lane;            // row within this CTA's 128 == TMEM lane
-    const uint32_t t_row = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kHalfN);
+    // One tile per unit (small K): the two warps of a lane quarter take
+    // alternate units whole, each on its own accumulator (unit u on u % 2),
+    // so a warp has two tiles of MMA time to read it and no merge is needed.
+    // Otherwise warp h takes columns [128h, 128h + 128) of every tile.
+    const bool whole = p.ntiles == 1;
+    const uint32_t t_row = tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(whole ? 0 : h * kHalfN);
     // hand an accumulator back to the leader's MMA thread
     auto release_acc = [&](int a) {
       if (leader) mbar_arrive(accempty(a));
       else mbar_arrive_cluster_relaxed(map_to_cta(accempty(a), 0));
     };
-    // Both accumulators start out free.
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-      release_acc(0);
-      release_acc(1);
-    }
-
-    uint32_t xb = 0, xc = 0;
-    int t = 0;  // the pair's tile counter
-    bool ok = true;
-    for (int u = u_begin; ok && u < u_end; ++u, xc ^= 1u) {
-      const int b = u / p.upb;
-      const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
-      Best bs;
-      bs.score = __int_as_float(0xff800000);
-      bs.base = 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
-      for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
-        const int a = t & 1;
-        if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
-        tc_fence_after();
-        if (h == 0 && q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
-        const uint32_t ta = t_row + a * kTileN;
-        const int col = j * kTileN + h * kHalfN;
-        uint32_t va[32], vb[32], vc[32];
-        // chunks 0 and 1; the loads of chunks 2 and 3 are issued while they
-        // are folded (chunk 3 into chunk 0's registers once it is folded)
-        FK_TMEM_LD32(ta, va);
-        FK_TMEM_LD32(ta + 32, vb);
-        FK_TMEM_WAIT_LD(va);
-        FK_TMEM_WAIT_LD(vb);
-        FK_TMEM_LD32(ta + 64, vc);
-        fold_chunk(bs, va, col);
-        FK_TMEM_LD32(ta + 96, va);
-        fold_chunk(bs, vb, col + 32);
-        // chunks 2 and 3: once they are in registers the accumulator is free
-        FK_TMEM_WAIT_LD(vc);
-        FK_TMEM_WAIT_LD(va);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) release_acc(a);
-        fold_chunk(bs, vc, col + 64);
-        fold_chunk(bs, va, col + 96);
-      }
-      if (!ok) break;
-      // lowest column of the candidate chunk holding the maximum
+    // lowest column of the candidate chunk holding the maximum
+    auto best_index = [&](const Best &bs) {
       int j0 = 32, j1 = 32, j2 = 32, j3 = 32;
 #pragma unroll
       for (int i = 28; i >= 0; i -= 4) {
@@ -456,64 +418,175 @@ __global__ void __launch_bounds__(kThreads, 1)
         j3 = __uint_as_float(bs.cand[i + 3]) == bs.score ? i + 3 : j3;
       }
       const int jm = min(min(j0, j1), min(j2, j3));
-      const int bi = jm < 32 ? bs.base + jm : 0;
-      // merge the two column halves of each point: half 1 hands over its
-      // candidate and |x|^2, half 0 merges and writes
-      if (h == 1) {
-        if (u != u_begin && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
-        float xn = 0.f;
-        if (p.mindist) {
-          // |x|^2 from the swizzled X tile: every MMA of this unit is done
-          // (its last accumulator was full), so X is resident until this
-          // CTA's epilogue warps have all arrived on xempty below
-          for (int kb = 0; kb < KB; ++kb) {
-            const uint8_t *rowp = sm + (xb * KB + kb) * kXBytes + r * 128;
+      return jm < 32 ? bs.base + jm : 0;
+    };
+    // |x|^2 of this thread's row from the swizzled X tile in buffer xb: every
+    // MMA of the unit is done (its last accumulator was full), so X is
+    // resident until this CTA's warps of the unit have arrived on xempty
+    auto x_norm = [&](uint32_t xb) {
+      float xn = 0.f;
+      for (int kb = 0; kb < KB; ++kb) {
+        const uint8_t *rowp = sm + (xb * KB + kb) * kXBytes + r * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint4 wv = *reinterpret_cast<const uint4 *>(rowp + ((c ^ (r & 7)) << 4));
-              const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+        for (int c = 0; c < 8; ++c) {
+          const uint4 wv = *reinterpret_cast<const uint4 *>(rowp + ((c ^ (r & 7)) << 4));
+          const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                float lo, hi;
-                if (p.is_bf16) {
-                  lo = __uint_as_float(ws[e] << 16);
-                  hi = __uint_as_float(ws[e] & 0xffff0000u);
-                } else {
-                  const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[e]);
-                  lo = __low2float(h2);
-                  hi = __high2float(h2);
-                }
-                xn = fmaf(lo, lo, xn);
-                xn = fmaf(hi, hi, xn);
-              }
+          for (int e = 0; e < 4; ++e) {
+            float lo, hi;
+            if (p.is_bf16) {
+              lo = __uint_as_float(ws[e] << 16);
+              hi = __uint_as_float(ws[e] & 0xffff0000u);
+            } else {
+              const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[e]);
+              lo = __low2float(h2);
+              hi = __high2float(h2);
             }
+            xn = fmaf(lo, lo, xn);
+            xn = fmaf(hi, hi, xn);
           }
         }
-        xchg[r] = make_float4(bs.score, __int_as_float(bi), xn, 0.f);
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(xchg_full);
-          mbar_arrive(xempty(xb));
-        }
+      }
+      return xn;
+    };
+    // The accumulators start out free.
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      if (whole) {
+        release_acc(h);
       } else {
-        if (!(ok = mbar_wait(xchg_full, xc, abort_flag, p.ctl))) break;
-        const float4 o = xchg[r];
-        float sb = bs.score;
-        int bb = bi;
-        const int oi = __float_as_int(o.y);
-        if (o.x > sb || (o.x == sb && oi < bb)) { sb = o.x; bb = oi; }
+        release_acc(0);
+        release_acc(1);
+      }
+    }
+
+    if (whole) {
+      bool ok = true;
+      for (int u = u_begin + h; ok && u < u_end; u += 2) {
+        const int t = u - u_begin, a = t & 1;  // a == h
+        const int b = u / p.upb;
+        const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
+        const uint32_t xb = (uint32_t)(t % XBUF);
+        Best bs;
+        bs.score = __int_as_float(0xff800000);
+        bs.base = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
+        if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
+        tc_fence_after();
+        if (q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
+        const uint32_t ta = t_row + a * kTileN;
+        uint32_t va[32], vb[32], vc[32];
+        // eight chunks; each load is issued while the chunk before is folded
+        FK_TMEM_LD32(ta, va);
+        FK_TMEM_LD32(ta + 32, vb);
+        FK_TMEM_WAIT_LD(va);
+        FK_TMEM_WAIT_LD(vb);
+        FK_TMEM_LD32(ta + 64, vc);
+        fold_chunk(bs, va, 0);
+        FK_TMEM_LD32(ta + 96, va);
+        fold_chunk(bs, vb, 32);
+        FK_TMEM_WAIT_LD(vc);
+        FK_TMEM_WAIT_LD(va);
+        FK_TMEM_LD32(ta + 128, vb);
+        fold_chunk(bs, vc, 64);
+        FK_TMEM_LD32(ta + 160, vc);
+        fold_chunk(bs, va, 96);
+        FK_TMEM_WAIT_LD(vb);
+        FK_TMEM_WAIT_LD(vc);
+        FK_TMEM_LD32(ta + 192, va);
+        fold_chunk(bs, vb, 128);
+        FK_TMEM_LD32(ta + 224, vb);
+        fold_chunk(bs, vc, 160);
+        FK_TMEM_WAIT_LD(va);
+        FK_TMEM_WAIT_LD(vb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release_acc(a);
+        fold_chunk(bs, va, 192);
+        fold_chunk(bs, vb, 224);
+        const int bi = best_index(bs);
         if (row < p.N) {
           const size_t o_ = (size_t)b * p.N + row;
-          p.labels[o_] = bb;
-          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, sb, o.z));
+          p.labels[o_] = bi;
+          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, bs.score, x_norm(xb)));
         }
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(xchg_empty);
-          mbar_arrive(xempty(xb));
-        }
+        if (lane == 0) mbar_arrive(xempty(xb));
       }
-      if (++xb == XBUF) xb = 0;
+    } else {
+      uint32_t xb = 0, xc = 0;
+      int t = 0;  // the pair's tile counter
+      bool ok = true;
+      for (int u = u_begin; ok && u < u_end; ++u, xc ^= 1u) {
+        const int b = u / p.upb;
+        const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
+        Best bs;
+        bs.score = __int_as_float(0xff800000);
+        bs.base = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
+        for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
+          const int a = t & 1;
+          if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
+          tc_fence_after();
+          if (h == 0 && q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
+          const uint32_t ta = t_row + a * kTileN;
+          const int col = j * kTileN + h * kHalfN;
+          uint32_t va[32], vb[32], vc[32];
+          // chunks 0 and 1; the loads of chunks 2 and 3 are issued while they
+          // are folded (chunk 3 into chunk 0's registers once it is folded)
+          FK_TMEM_LD32(ta, va);
+          FK_TMEM_LD32(ta + 32, vb);
+          FK_TMEM_WAIT_LD(va);
+          FK_TMEM_WAIT_LD(vb);
+          FK_TMEM_LD32(ta + 64, vc);
+          fold_chunk(bs, va, col);
+          FK_TMEM_LD32(ta + 96, va);
+          fold_chunk(bs, vb, col + 32);
+          // chunks 2 and 3: once they are in registers the accumulator is free
+          FK_TMEM_WAIT_LD(vc);
+          FK_TMEM_WAIT_LD(va);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release_acc(a);
+          fold_chunk(bs, vc, col + 64);
+          fold_chunk(bs, va, col + 96);
+        }
+        if (!ok) break;
+        const int bi = best_index(bs);
+        // merge the two column halves of each point: half 1 hands over its
+        // candidate and |x|^2, half 0 merges and writes
+        if (h == 1) {
+          if (u != u_begin && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
+          const float xn = p.mindist ? x_norm(xb) : 0.f;
+          xchg[r] = make_float4(bs.score, __int_as_float(bi), xn, 0.f);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(xchg_full);
+            mbar_arrive(xempty(xb));
+          }
+        } else {
+          if (!(ok = mbar_wait(xchg_full, xc, abort_flag, p.ctl))) break;
+          const float4 o = xchg[r];
+          float sb = bs.score;
+          int bb = bi;
+          const int oi = __float_as_int(o.y);
+          if (o.x > sb || (o.x == sb && oi < bb)) { sb = o.x; bb = oi; }
+          if (row < p.N) {
+            const size_t o_ = (size_t)b * p.N + row;
+            p.labels[o_] = bb;
+            if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, sb, o.z));
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(xchg_empty);
+            mbar_arrive(xempty(xb));
+          }
+        }
+        if (++xb == XBUF) xb = 0;
+      }
     }
   }
 

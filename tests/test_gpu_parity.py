@@ -62,16 +62,20 @@ def test_tensor_and_cuda_core_paths_agree(dtype):
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 @pytest.mark.parametrize("path", [1, 2])
-def test_integer_inputs_bit_exact_with_ties(dtype, path):
+@pytest.mark.parametrize("K", [300, 200])
+def test_integer_inputs_bit_exact_with_ties(dtype, path, K):
     """Small integers: products and fp32 sums are exact, so labels (including
-    lowest-index tie-breaks on duplicated centroids) and mindist are exact."""
+    lowest-index tie-breaks on duplicated centroids) and mindist are exact.
+    K = 200 fits one 256-centroid tile (each point's whole row of scores is
+    read by one warp); K = 300 spans two."""
     if dtype == "f32" and path == 1:
         pytest.skip("fp32 runs on the CUDA-core kernel only")
     g = torch.Generator().manual_seed(5)
-    N, D, K = 3000, 64, 300
+    N, D = 3000, 64
+    third = K // 3
     X = torch.randint(-8, 9, (N, D), generator=g).to(TORCH_DT[dtype])
-    C = torch.cat([X[:100], X[:100], torch.randint(-8, 9, (100, D), generator=g).to(TORCH_DT[dtype])])
-    C[250] = C[10]  # later duplicate of an earlier centroid
+    C = torch.cat([X[:third], X[:third], torch.randint(-8, 9, (K - 2 * third, D), generator=g).to(TORCH_DT[dtype])])
+    C[K - 50] = C[10]  # later duplicate of an earlier centroid
     try:
         fk.fk_set_assign_path(path)
         labels, mind = fk.fk_assign(X.to(DEV), C.to(DEV), want_mindist=True)
@@ -81,11 +85,12 @@ def test_integer_inputs_bit_exact_with_ties(dtype, path):
     lab, md, _ = oracle.assign(f64(X), f64(C))
     assert np.array_equal(labels.cpu().numpy(), lab)
     assert np.array_equal(mind.cpu().numpy().astype(np.float64), md)
-    assert labels[:100].cpu().tolist() == list(range(100))
+    assert labels[:third].cpu().tolist() == list(range(third))
 
 
-def test_assign_batched_matches_per_problem():
-    B, N, D, K = 5, 1500, 128, 300
+@pytest.mark.parametrize("K", [300, 256])
+def test_assign_batched_matches_per_problem(K):
+    B, N, D = 5, 1500, 128
     s = workloads.spec("batched_bf16", N=N, K=K, n_centers=64, B=B)
     w = workloads.make(s, seed=1)
     X, C = w.X, w.C0.to(torch.bfloat16)
