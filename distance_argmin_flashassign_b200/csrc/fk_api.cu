@@ -275,7 +275,7 @@ fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t
   if (!X || !labels) return fail(FK_ERR_INVALID_ARG, "X and labels must not be NULL");
   DevState *d;
   if ((st = device_state(&d)) != FK_OK) return st;
-  const size_t need = update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D);
+  const size_t need = update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D, B);
   void *ws = nullptr;
   if ((st = scratch(*d, s, need, &ws)) != FK_OK) return st;
   UpdateArgs a{};
@@ -312,7 +312,7 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   if ((st = device_state(&d)) != FK_OK) return st;
   const DType t = (DType)dt;
   const int Kpad = pad_k(K);
-  const size_t upd = al256(update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D));
+  const size_t upd = al256(update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D, B));
   const size_t cnb = al256(bias_bytes(B, K));
   const size_t cdb = t == kF32 ? 0 : al256((size_t)B * K * D * dtype_size(t));
   void *ws = nullptr;
@@ -376,7 +376,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   const size_t b_c32 = al256((size_t)K * D * 4), b_cdt = t == kF32 ? 0 : al256((size_t)K * D * es);
   const size_t b_cn = al256(bias_bytes(1, K)), b_acc = al256((size_t)K * D * 8);
   const size_t b_cnt = al256((size_t)K * 8), b_counts = al256((size_t)K * 4);
-  const size_t b_upd = al256(update_workspace_bytes(rows, K, D));
+  const size_t b_upd = al256(update_workspace_bytes(rows, K, D, 1));
   const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd;
 
   Scratch *sc = nullptr;

@@ -57,7 +57,9 @@ struct UpdateArgs {
   long long *cnt;         // kAccumulate: B*K running counts
   UpdateMode mode;
 };
-size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D);
+// Device workspace of launch_update for B problems of Ntot / B points and
+// Ktot / B clusters each.
+size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D, int B);
 cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl ctl,
                           int num_sms, cudaStream_t s);
 // C[k] = acc[k] / cnt[k] (fp32) where cnt[k] > 0, counts[k] = cnt[k]; acc and

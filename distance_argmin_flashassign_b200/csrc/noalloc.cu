@@ -52,7 +52,7 @@ extern "C" fk_status fk_update_noalloc(const void *X, const int32_t *labels, int
     return FK_OK;
   }
   if (!X || !labels) return record_error(FK_ERR_INVALID_ARG, "X and labels must not be NULL");
-  const size_t need = update_workspace_bytes(N, K, D);
+  const size_t need = update_workspace_bytes(N, K, D, 1);
   if (need > kNoAllocScratchBytes - kNoAllocStatusBytes) {
     const std::string msg = "fk_update_noalloc needs " + std::to_string(need) +
                             " bytes of scratch; its static scratch holds " +

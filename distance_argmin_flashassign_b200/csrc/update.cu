@@ -60,7 +60,8 @@ constexpr int kMaxBins = 1 << kMaxDigitBits;
 struct SortPlan {
   int npass;
   int shift[2], bits[2];
-  int T;  // tiles
+  int T;          // tiles
+  int seg_tiles;  // > 0: one pass on the label digit, problems of seg_tiles whole tiles each
 };
 
 static int ceil_log2(long long v) {
@@ -69,7 +70,12 @@ static int ceil_log2(long long v) {
   return b;
 }
 
-static SortPlan plan_sort(long long Ntot, long long Ktot) {
+// A batch of B problems whose N is a whole number of tiles is sorted in one
+// pass on the label alone when the key b*K + label would need two: the
+// problems' points are already in problem order, and each tile belongs to
+// one problem, so ranking a tile's points by label and placing problem b's
+// runs at b*N gives the order of a stable sort by key.
+static SortPlan plan_sort(long long Ntot, long long Ktot, int B) {
   SortPlan p{};
   int bits = ceil_log2(Ktot);
   if (bits < 1) bits = 1;
@@ -82,6 +88,12 @@ static SortPlan plan_sort(long long Ntot, long long Ktot) {
     sh += p.bits[i];
   }
   p.T = (int)((Ntot + kSortTile - 1) / kSortTile);
+  if (B > 1 && p.npass > 1 && (Ntot / B) % kSortTile == 0 && ceil_log2(Ktot / B) <= kMaxDigitBits) {
+    p.npass = 1;
+    p.shift[0] = 0;
+    p.bits[0] = ceil_log2(Ktot / B) < 1 ? 1 : ceil_log2(Ktot / B);
+    p.seg_tiles = (int)(Ntot / B / kSortTile);
+  }
   return p;
 }
 
@@ -111,11 +123,12 @@ __device__ __forceinline__ int key_of_label(int lab, int pos, int N, int K, int 
   return B > 1 ? (pos / N) * K + lab : lab;
 }
 
-template <bool FIRST>
+// SEG: one pass per problem (the digit is the label), see plan_sort.
+template <bool FIRST, bool SEG>
 __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t *__restrict__ keys, int Ntot,
                                                                   int N, int K, int B, int shift, int nbins,
                                                                   int T, int *__restrict__ H,
-                                                                  int *status) {
+                                                                  int *status, int seg_tiles) {
   __shared__ int hist[kMaxBins + 1];
   for (int i = threadIdx.x; i <= nbins; i += kSortThreads) hist[i] = 0;
   __syncthreads();
@@ -136,7 +149,8 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(const int32_t 
     int d = nbins;  // spare bin for positions past the end
     if (pos < Ntot) {
       const int key = FIRST ? key_of_label(v[it], pos, N, K, B, bad) : v[it];
-      d = (key >> shift) & (nbins - 1);
+      // one pass per problem: the digit is the label (each tile lies in one problem)
+      d = SEG ? key - ((int)blockIdx.x / seg_tiles) * K : (key >> shift) & (nbins - 1);
     }
     atomicAdd(&hist[d], 1);
   }
@@ -188,11 +202,11 @@ static size_t scatter_smem_bytes(int nbins) {
   return (size_t)(2 * nbins + kSortWarps + scatter_xbuf_ints(nbins)) * 4 + (size_t)kSortWarps * (nbins + 1) * 4;
 }
 
-template <bool FIRST>
+template <bool FIRST, bool SEG>
 __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     const int32_t *__restrict__ keys_in, const int32_t *__restrict__ vals_in, int32_t *__restrict__ keys_out,
     int32_t *__restrict__ vals_out, int Ntot, int N, int K, int B, int shift, int nbins, int T,
-    const int *__restrict__ H, const int *__restrict__ totals, int *status) {
+    const int *__restrict__ H, const int *__restrict__ totals, int *status, int seg_tiles) {
   extern __shared__ int sh[];
   const int stride = nbins + 1;
   int *dbase = sh;                                                   // [nbins]
@@ -203,6 +217,10 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   unsigned *wmask = reinterpret_cast<unsigned *>(keys_s);            // [kSortWarps][nbins], same place
   int *wcnt = keys_s + scatter_xbuf_ints(nbins);                     // [kSortWarps][nbins + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // one pass per problem (SEG): this tile's problem; the digit is the label
+  // and the problem's runs start at pb * N
+  const int pb = SEG ? (int)blockIdx.x / seg_tiles : 0;
+  auto digit = [&](int key) { return SEG ? key - pb * K : (key >> shift) & (nbins - 1); };
   wait_prior_grid();
   // the warp's 512 consecutive keys and values are loaded first, so that
   // their latency overlaps the digit-base reads below
@@ -224,8 +242,18 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   for (int i = 0; i < kPer; ++i) {
     const int d = tid * per + i;
     const bool ok = i < per && d < nbins;
-    tv[i] = ok ? totals[d] : 0;
-    hv[i] = ok ? H[(size_t)d * T + blockIdx.x] : 0;
+    if (SEG) {
+      // the problem's count of digit d and the count in its tiles before
+      // this one, from the prefix over all tiles at the problem's bounds
+      const int t0 = pb * seg_tiles, t1 = t0 + seg_tiles;
+      const int p0 = ok ? H[(size_t)d * T + t0] : 0;
+      const int p1 = ok ? (t1 < T ? H[(size_t)d * T + t1] : totals[d]) : 0;
+      tv[i] = p1 - p0;
+      hv[i] = (ok ? H[(size_t)d * T + blockIdx.x] : 0) - p0;
+    } else {
+      tv[i] = ok ? totals[d] : 0;
+      hv[i] = ok ? H[(size_t)d * T + blockIdx.x] : 0;
+    }
   }
   int s = 0;
 #pragma unroll
@@ -240,7 +268,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   for (int i = tid; i < kSortWarps * stride; i += kSortThreads) wcnt[i] = 0;
   for (int i = tid; i < kSortWarps * nbins; i += kSortThreads) wmask[i] = 0u;
   __syncthreads();
-  int run = incl - s;
+  int run = incl - s + pb * N;
   for (int w = 0; w < warp; ++w) run += wsum[w];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
@@ -269,7 +297,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     int d = 0;
     if (valid) {
       if (FIRST) keyr[it] = key_of_label(keyr[it], pos, N, K, B, bad);
-      d = (keyr[it] >> shift) & (nbins - 1);
+      d = digit(keyr[it]);
     }
     if (valid) atomicOr(mymask + d, 1u << lane);
     __syncwarp();
@@ -328,7 +356,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
   for (int it = 0; it < kSortItems; ++it) {
     const int pos = base + it * 32 + lane;
     if (pos < Ntot) {
-      const int d = (keyr[it] >> shift) & (nbins - 1);
+      const int d = digit(keyr[it]);
       const int lp = tstart[d] + mycnt[d] + locr[it];
       keys_s[lp] = keyr[it];
       vals_s[lp] = valr[it];
@@ -343,7 +371,7 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     const int idx = it * kSortThreads + tid;
     if (idx < nvalid) {
       const int key = keys_s[idx];
-      const int d = (key >> shift) & (nbins - 1);
+      const int d = digit(key);
       const int o = dbase[d] + (idx - tstart[d]);
       keys_out[o] = key;
       vals_out[o] = vals_s[idx];
@@ -912,8 +940,8 @@ struct UpdateWs {
   size_t bytes;
 };
 
-static UpdateWs carve(void *base, long long Ntot, long long Ktot, int D) {
-  const SortPlan sp = plan_sort(Ntot, Ktot);
+static UpdateWs carve(void *base, long long Ntot, long long Ktot, int D, int B) {
+  const SortPlan sp = plan_sort(Ntot, Ktot, B);
   const int R = chunk_rows_R(Ntot);
   const long long nchunks = (Ntot + R - 1) / R;
   int maxbins = 0;
@@ -934,8 +962,8 @@ static UpdateWs carve(void *base, long long Ntot, long long Ktot, int D) {
   return w;
 }
 
-size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D) {
-  return carve(nullptr, Ntot, Ktot, D).bytes;
+size_t update_workspace_bytes(int64_t Ntot, int64_t Ktot, int D, int B) {
+  return carve(nullptr, Ntot, Ktot, D, B).bytes;
 }
 
 template <typename T, int MODE, int NACC>
@@ -1008,9 +1036,9 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
                           cudaStream_t s) {
   const long long Ntot = (long long)a.B * a.N, Ktot = (long long)a.B * a.K;
   if (Ntot == 0) return cudaSuccess;
-  const UpdateWs w = carve(ws, Ntot, Ktot, a.D);
+  const UpdateWs w = carve(ws, Ntot, Ktot, a.D, a.B);
   if (w.bytes > ws_bytes) return cudaErrorInvalidValue;
-  const SortPlan sp = plan_sort(Ntot, Ktot);
+  const SortPlan sp = plan_sort(Ntot, Ktot, a.B);
   const int N = (int)Ntot;
   int nl = 0;
 
@@ -1020,8 +1048,9 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
     cudaGetDevice(&dev);
     if (dev < 64 && !configured[dev]) {
       const int most = (int)scatter_smem_bytes(kMaxBins);
-      cudaFuncSetAttribute(radix_scatter_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-      cudaFuncSetAttribute(radix_scatter_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(radix_scatter_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(radix_scatter_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(radix_scatter_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
       configured[dev] = true;
     }
   }
@@ -1029,22 +1058,16 @@ cudaError_t launch_update(const UpdateArgs &a, void *ws, size_t ws_bytes, DevCtl
   int32_t *kout = w.kA, *vout = w.vA;
   for (int pass = 0; pass < sp.npass; ++pass) {
     const int nbins = 1 << sp.bits[pass];
-    if (pass == 0)
-      launch_chained(radix_hist_kernel<true>, dim3(sp.T), dim3(kSortThreads), 0, s, kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
-                                                            sp.T, w.H, ctl.status);
-    else
-      launch_chained(radix_hist_kernel<false>, dim3(sp.T), dim3(kSortThreads), 0, s, kin, N, a.N, a.K, a.B, sp.shift[pass], nbins,
-                                                             sp.T, w.H, ctl.status);
+    const bool seg = sp.seg_tiles > 0;  // one pass, so pass == 0
+    const auto hist = pass > 0 ? radix_hist_kernel<false, false> : seg ? radix_hist_kernel<true, true>
+                                                                          : radix_hist_kernel<true, false>;
+    launch_chained(hist, dim3(sp.T), dim3(kSortThreads), 0, s, kin, N, a.N, a.K, a.B, sp.shift[pass], nbins, sp.T, w.H,
+                   ctl.status, sp.seg_tiles);
     launch_chained(scan_rows_kernel, dim3((nbins + 7) / 8), dim3(256), 0, s, w.H, sp.T, nbins, w.totals);
-    const size_t shb = scatter_smem_bytes(nbins);
-    if (pass == 0)
-      launch_chained(radix_scatter_kernel<true>, dim3(sp.T), dim3(kSortThreads), shb, s, kin, vin, kout, vout, N, a.N, a.K, a.B,
-                                                                 sp.shift[pass], nbins, sp.T, w.H,
-                                                                 w.totals, ctl.status);
-    else
-      launch_chained(radix_scatter_kernel<false>, dim3(sp.T), dim3(kSortThreads), shb, s, kin, vin, kout, vout, N, a.N, a.K, a.B,
-                                                                  sp.shift[pass], nbins, sp.T, w.H,
-                                                                  w.totals, ctl.status);
+    const auto scatter = pass > 0 ? radix_scatter_kernel<false, false>
+                                  : seg ? radix_scatter_kernel<true, true> : radix_scatter_kernel<true, false>;
+    launch_chained(scatter, dim3(sp.T), dim3(kSortThreads), scatter_smem_bytes(nbins), s, kin, vin, kout, vout, N, a.N,
+                   a.K, a.B, sp.shift[pass], nbins, sp.T, w.H, w.totals, ctl.status, sp.seg_tiles);
     nl += 3;
     kin = kout;
     vin = vout;

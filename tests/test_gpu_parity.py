@@ -133,11 +133,16 @@ def test_update_is_deterministic():
     assert torch.equal(outs[0], outs[1])
 
 
-def test_update_batched():
-    B, N, D, K = 4, 3000, 64, 500
+@pytest.mark.parametrize("B,N,D,K,kind", [
+    (4, 3000, 64, 500, "zipf"),       # B*K fits one 11-bit sort pass
+    (4, 8192, 64, 1000, "zipf"),      # B*K needs two passes; N is whole sort tiles: one pass per problem
+    (3, 12288, 32, 700, "uniform"),   # the same with K not a power of two
+    (3, 5000, 32, 1000, "uniform"),   # two passes; N not whole tiles: the two-pass sort
+])
+def test_update_batched(B, N, D, K, kind):
     s = workloads.spec("batched_bf16", N=N, D=D, K=K, n_centers=50, B=B)
     X = workloads.make(s, seed=2).X
-    labels = torch.stack([workloads.labels(N, K, seed=b, kind="zipf") for b in range(B)])
+    labels = torch.stack([workloads.labels(N, K, seed=b, kind=kind) for b in range(B)])
     C = torch.zeros(B, K, D, device=DEV)
     counts = torch.empty(B, K, dtype=torch.int32, device=DEV)
     fk.fk_update(X.to(DEV), labels.to(DEV), C, counts)
@@ -158,6 +163,22 @@ def test_update_reports_bad_label():
         fk.fk_sync()
     assert e.value.status == fk.FK_ERR_BAD_LABEL
     fk.fk_sync()  # the status word was cleared
+
+
+def test_update_batched_reports_bad_label():
+    B, N, D, K = 2, 4096, 16, 1500  # sorted in one pass per problem
+    X = torch.randn(B, N, D, device=DEV)
+    labels = torch.zeros(B, N, dtype=torch.int32, device=DEV)
+    labels[1, 17] = K + 3
+    C = torch.zeros(B, K, D, device=DEV)
+    counts = torch.empty(B, K, dtype=torch.int32, device=DEV)
+    fk.fk_update(X, labels, C, counts)
+    with pytest.raises(fk.FKError) as e:
+        fk.fk_sync()
+    assert e.value.status == fk.FK_ERR_BAD_LABEL
+    # the bad label was counted in its problem's cluster 0
+    assert counts[0, 0].item() == N and counts[1, 0].item() == N
+    fk.fk_sync()
 
 
 LLOYD_CASES = [
