@@ -13,7 +13,12 @@ all through the C ABI, inputs resident in HBM (X = 256 MiB, larger than the
 126 MB L2, so no flush is needed between steps).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu]
+                    [--workload NAME] [--no-e2e] [--no-cpu] [--ooc-rows R]
+
+--workload ooc_f16 runs the out-of-core workload instead (one GPU): X in
+pinned host memory, streamed through fk_lloyd_ooc in the configured 64 Mi-row
+chunks, --ooc-rows rows (the configured 10^9 rows need 256 GB of pinned host
+memory, more than the host has).
 
 Prints one JSON line (rank 0).  Multi-GPU runs are replicas: every rank runs
 its own copy of the workload, there is no collective on the data path, the
@@ -344,6 +349,103 @@ def bench_e2e(args, s, w, fk, dev, world):
             "api": "fk_lloyd_ooc(iters=1, chunk_rows=N/4), pinned host X"}
 
 
+# ---------------------------------------------------------- out of core --
+def ooc_inputs(rows: int, device):
+    """X of the out-of-core workload with ``rows`` rows in pinned host memory
+    (generated on the device block by block, same recipe as the full
+    workload's first rows), and its configured initial centroids."""
+    import torch
+
+    import workloads
+    s = workloads.spec("ooc_f16", N=rows)
+    Xh = torch.empty((rows, s.D), dtype=torch.float16, pin_memory=True)
+    cen = workloads.centers(s, 0, device)
+    piece = 1 << 24
+    for r0 in range(0, rows, piece):
+        Xh[r0:r0 + piece].copy_(workloads.rows(s, r0, min(rows, r0 + piece), device=device, cen=cen))
+    return s, Xh, Xh[: s.K].float().clone()  # init = first K rows
+
+
+def bench_ooc(args):
+    """The configured iterations of the out-of-core workload in one
+    fk_lloyd_ooc call: every chunk of X crosses the host link once per
+    iteration on a copy stream while the previous chunk is assigned and
+    accumulated.  The host-to-device rate is reported against a plain copy
+    of one chunk from the same pinned buffer, timed in this process."""
+    import torch
+
+    import distance_argmin_flashassign_b200 as fk
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit("ooc_f16 runs on one GPU (its pinned host copy of X does not fit once per rank)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    s, Xh, C0 = ooc_inputs(args.ooc_rows, dev)
+    N, D, K, chunk, iters = s.N, s.D, s.K, s.chunk_rows, s.iters
+    stream = torch.cuda.current_stream(dev)
+    # the plain pinned-to-device copy rate of one chunk
+    dchunk = torch.empty((min(chunk, N), D), dtype=torch.float16, device=dev)
+    dchunk.copy_(Xh[: dchunk.shape[0]], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        dchunk.copy_(Xh[: dchunk.shape[0]], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    copy_gbs = 3 * dchunk.numel() * 2 / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del dchunk
+    torch.cuda.empty_cache()
+
+    lab_h = torch.empty(N, dtype=torch.int32, pin_memory=True)
+    cnt_h = torch.empty(K, dtype=torch.int32)
+    Ch = C0.clone()
+    fk.fk_lloyd_ooc(Xh, Ch, 1, chunk, lab_h, cnt_h)  # warm-up: sets up the device ring and workspace
+    torch.cuda.synchronize(dev)
+    Ch = C0.clone()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = fk.fk_launch_count()
+    w0 = time.time()
+    e0.record(stream)
+    fk.fk_lloyd_ooc(Xh, Ch, iters, chunk, lab_h, cnt_h)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    launches = fk.fk_launch_count() - n0
+    clocks.stop()
+    ms = e0.elapsed_time(e1)
+    value = iters / (ms * 1e-3)
+    h2d_gbs = iters * N * D * 2 / (ms * 1e-3) / 1e9
+    nchunks = (N + chunk - 1) // chunk
+    out = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1, "steps": iters,
+           "warmup": 1, "ms_per_step": round(ms / iters, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+           "config": {"workload": "ooc_f16", "N": N, "N_configured": 10 ** 9, "D": D, "K": K, "B": 1,
+                      "dtype": s.dtype, "chunk_rows": chunk, "chunks_per_iteration": nchunks,
+                      "step": "one Lloyd iteration streamed from pinned host memory (fk_lloyd_ooc, "
+                              f"{iters} iterations in one call)",
+                      "reduced_N": "the configured 10^9 rows need 256 GB of pinned host memory"},
+           "roofline": {"bound": "host-to-device copy", "achieved": round(h2d_gbs, 2),
+                        "peak": round(copy_gbs, 2), "unit": "GB/s", "frac": round(h2d_gbs / copy_gbs, 4),
+                        "peak_kind": "plain copy of one chunk from the same pinned buffer, measured in this run",
+                        "traffic": None},
+           "gpu_launches": launches, "clocks": clocks.summary(w0, w1),
+           "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": N * D * 2 + K * D * 4,
+                   "d2h_bytes_per_step": K * D * 4 + K * 4 + (N * 4) // iters}}
+    if args.cpu:
+        import workloads
+        n = min(N, 1 << 16)
+        Xs = workloads.rows(s, 0, n, device=dev).cpu()
+        v, n_used, reps, secs, cores = oracle_throughput(Xs.double().numpy(), C0.double().numpy(), s.dtype, N,
+                                                         args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(v, 8), "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{reps} x {n_used} of {N} rows against all {K} centroids, one Lloyd "
+                                         f"step each ({secs:.1f} s in all), scaled linearly in N"}
+    print(json.dumps(out), flush=True)
+
+
 # -------------------------------------------------------- reference arm --
 def bench_reference(args):
     """The oracle, as it stands, on the host cores: each step is one Lloyd
@@ -357,9 +459,14 @@ def bench_reference(args):
     import workloads
     s = workloads.spec(args.workload)
     per_step = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
-    w = workloads.make(s.replace(B=1) if s.B > 1 else s, seed=0, device="cpu")
-    X64 = w.X.double().numpy()
-    C64 = w.C0.double().numpy()
+    if s.name == "ooc_f16":  # the same reduced N as the own arm; a row sample only
+        s = s.replace(N=args.ooc_rows)
+        X64 = workloads.rows(s, 0, min(s.N, 1 << 16)).double().numpy()
+        C64 = X64[: s.K].copy()
+    else:
+        w = workloads.make(s.replace(B=1) if s.B > 1 else s, seed=0, device="cpu")
+        X64 = w.X.double().numpy()
+        C64 = w.C0.double().numpy()
     import oracle
     lib = oracle.load()
     t = time.perf_counter()
@@ -399,10 +506,14 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
+    ap.add_argument("--ooc-rows", type=int, default=1 << 28,
+                    help="rows of the out-of-core workload (default 2^28: 64 GiB of pinned fp16, 4 chunks)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps, reported as run
     if args.impl == "reference":
         bench_reference(args)
+    elif args.workload == "ooc_f16":
+        bench_ooc(args)
     else:
         bench_gpu(args)
 
