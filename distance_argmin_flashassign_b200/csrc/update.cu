@@ -872,17 +872,25 @@ __global__ void __launch_bounds__(1024) seg_finalize_kernel(const int *__restric
         if (lane == 0) hot[atomicAdd(&nhot, 1)] = k;
         continue;
       }
-      // 4 dimensions per lane per pass; every partial row's loads are
-      // independent of the running sums, so they are all in flight together
+      // 4 dimensions per lane per pass; the partial rows are loaded 4 at a
+      // time (in flight together), then added in chunk order
       for (int d0 = 0; d0 < D; d0 += 128) {
         float t[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int i = 0; i < np; ++i) {
-          const float *row = part_row(s, q0, i) + d0;
-          float v[4];
+        for (int i0 = 0; i0 < np; i0 += 4) {
+          float v[4][4];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) v[jj] = d0 + lane + 32 * jj < D ? row[lane + 32 * jj] : 0.f;
+          for (int ii = 0; ii < 4; ++ii) {
+            const bool in = i0 + ii < np;
+            const float *row = part_row(s, q0, in ? i0 + ii : 0) + d0;
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) t[jj] += v[jj];
+            for (int jj = 0; jj < 4; ++jj) v[ii][jj] = in && d0 + lane + 32 * jj < D ? row[lane + 32 * jj] : 0.f;
+          }
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+            if (i0 + ii < np) {
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) t[jj] += v[ii][jj];
+            }
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
@@ -897,11 +905,23 @@ __global__ void __launch_bounds__(1024) seg_finalize_kernel(const int *__restric
       const int q0 = s / R, np = (e - 1) / R - q0 + 1;
       for (int d0 = 0; d0 < D; d0 += 128) {
         float t[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int i = w; i < np; i += 32) {
-          const float *row = part_row(s, q0, i) + d0;
+        // rows w, w + 32, ... in that order, four loaded at a time
+        for (int i0 = w; i0 < np; i0 += 4 * 32) {
+          float v[4][4];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            if (d0 + lane + 32 * jj < D) t[jj] += row[lane + 32 * jj];
+          for (int ii = 0; ii < 4; ++ii) {
+            const int i = i0 + 32 * ii;
+            const float *row = part_row(s, q0, i < np ? i : 0) + d0;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) v[ii][jj] = i < np && d0 + lane + 32 * jj < D ? row[lane + 32 * jj] : 0.f;
+          }
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii)
+            if (i0 + 32 * ii < np) {
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+                if (d0 + lane + 32 * jj < D) t[jj] += v[ii][jj];
+            }
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) red[w][lane + 32 * jj] = t[jj];
