@@ -5,18 +5,20 @@
 // segment-level localized reductions.  Here:
 //
 //   1. stable LSD radix sort of the cluster ids (11-bit digits, one pass for
-//      up to 2,048 clusters, two for up to 2^22): per-tile digit histograms,
-//      a per-digit scan over tiles, and a scatter whose within-tile ranks come
-//      from warp ballots -- the sorted point ids are the inverse map
-//      (cluster -> its points);
+//      up to 2,048 clusters, two for up to 2^22; a batch of problems whose N
+//      is whole 4096-key tiles takes one pass on the label per problem):
+//      per-tile digit histograms, a per-digit scan over tiles, and a scatter
+//      whose within-tile ranks come from shared-memory digit masks -- the
+//      sorted point ids are the inverse map (cluster -> its points);
 //   2. segmented sums: the sorted order is cut into equal chunks of R
-//      positions, one warp per chunk, so a hot cluster (Zipf skew) is spread
-//      over many warps instead of serialising on one address.  A warp gathers
-//      its rows coalesced (each row is read as one contiguous vector per
-//      lane), accumulates in fp32 registers and writes a segment that lies
-//      wholly inside its chunk straight to the output; the two boundary
-//      segments of a chunk go to partial slots.  The same warps write the
-//      segment offsets (first sorted position of every cluster id);
+//      positions, one worker per chunk (a half warp for 256-byte rows), so a
+//      hot cluster (Zipf skew) is spread over many workers instead of
+//      serialising on one address.  A worker gathers its rows (each row read
+//      as one contiguous vector across its lanes), accumulates in fp32
+//      registers and writes a segment that lies wholly inside its chunk
+//      straight to the output; the two boundary segments of a chunk go to
+//      partial slots.  The same workers write the segment offsets (first
+//      sorted position of every cluster id);
 //   3. finalize: per cluster, partials of chunk-crossing segments are summed
 //      in a fixed order and divided by the count; empty clusters are left
 //      untouched.  No global atomics anywhere, so results are deterministic.
