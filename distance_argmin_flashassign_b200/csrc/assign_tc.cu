@@ -7,11 +7,13 @@
 //
 //   * clusters of two CTAs (one per SM) loop over "units" of 256 points; the
 //     leader CTA owns rows [0,128) of a unit, the peer rows [128,256);
-//   * in each CTA a TMA warp loads its 128 rows of X once per unit (kept
-//     resident while every centroid tile streams past) and, per 256-centroid
-//     tile, its half (128 centroids) into a ring of tile slots: the k-blocks
-//     of the centroids (128-byte swizzle, 64 elements each) and their bias
-//     terms (32-byte rows: three tf32-exact terms of -|c|^2/2, then zeros);
+//   * in each CTA one TMA warp streams its 128 rows of X per unit into a ring
+//     of X buffers (kept resident while every centroid tile streams past;
+//     deeper when a unit has at most two tiles), and another loads, per
+//     256-centroid tile, its half (128 centroids) into a ring of tile slots:
+//     the k-blocks of the centroids (128-byte swizzle, 64 elements each) and
+//     their bias terms (32-byte rows: three tf32-exact terms of -|c|^2/2,
+//     then zeros); a slot that already holds the wanted tile is reused;
 //   * one thread of the leader issues the tile's MMAs with cta_group::2
 //     (M = 256 across the pair, N = 256, fp32 accumulate; each CTA's TMEM
 //     receives its 128 rows x 256 columns).  The first, of kind tf32 and
@@ -29,7 +31,9 @@
 //     complete, and a unit's X buffer once it is done with the unit;
 //   * eight epilogue warps per CTA: warp (h, q) owns TMEM lanes [32q, 32q+32)
 //     (one point per thread) and columns [128h, 128h+128) of every tile, read
-//     as two pairs of 32-column chunks.  A 3-input-max tree gives the chunk
+//     as two pairs of 32-column chunks (with one tile per unit, warp (h, q)
+//     instead takes every other unit whole, on accumulator h, and no merge
+//     is needed).  A 3-input-max tree gives the chunk
 //     maximum; when it beats the point's running maximum (strict
 //     ">", so an earlier column keeps a tie) the lane copies the chunk into a
 //     register-resident candidate.  The lowest column of the candidate
@@ -37,9 +41,9 @@
 //     of a point are merged at the end of the unit (score, then lower index),
 //     together with |x|^2 for the returned squared distance;
 //   * nothing is written back to TMEM, so an accumulator goes back to the MMA
-//     thread as soon as all 16 epilogue warps of the pair have LOADED their
-//     last chunk pair: the reduction of that pair overlaps the next tile's
-//     MMAs.  The peer's warps signal the leader's barrier with a relaxed
+//     thread as soon as all epilogue warps of the pair that read it have
+//     LOADED their last chunk pair (issued while the pair before it is
+//     folded): the reduction of that pair overlaps the next tile's MMAs.  The peer's warps signal the leader's barrier with a relaxed
 //     cluster-scope arrive, after tcgen05.wait::ld and
 //     tcgen05.fence::before_thread_sync: a release at cluster scope would cost
 //     more than a third of a tile, and those TMEM reads are already complete
