@@ -66,6 +66,15 @@ def test_reference_arm_json_line():
     assert line["config"]["workload"] == "tiny_f32"
 
 
+def test_reference_arm_out_of_core_uses_the_reduced_rows():
+    out = _run_bench(["--impl", "reference", "--steps", "3", "--warmup", "3", "--workload", "ooc_f16",
+                      "--ref-budget", "1", "--ooc-rows", str(1 << 20)])
+    line = json.loads(out.strip().splitlines()[-1])
+    cfg = line["config"]
+    assert cfg["workload"] == "ooc_f16" and cfg["N"] == 1 << 20 and cfg["K"] == 8192 and cfg["D"] == 128
+    assert line["impl"] == "reference" and line["value"] > 0
+
+
 def test_reference_arm_only_rank0_prints():
     out = _run_bench(["--impl", "reference", "--steps", "3", "--warmup", "3", "--workload", "tiny_f32",
                       "--ref-budget", "1"], {"RANK": "1", "WORLD_SIZE": "2"})
