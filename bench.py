@@ -44,6 +44,10 @@ if ROOT not in sys.path:
 
 METRIC = "k-means Lloyd iter/s; assign TFLOP/s & update GB/s as % of B200 roofline"
 UNIT = "iter/s"
+# FP32 lanes per SM and the maximum SM clock of a B200 (clocks.max.sm), for the
+# roofline of the fp32 CUDA-core assign kernel
+FP32_LANES_PER_SM = 128
+SM_MAX_GHZ = 1.965
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -279,11 +283,23 @@ def bench_gpu(args):
     upd_bytes = B * (N * D * es + 4 * N + K * (4 * D + 4))
     tflops = flops / (t_assign * 1e-3) / 1e12
     gbs = upd_bytes / (t_update * 1e-3) / 1e9
-    roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": round(tflops, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4),
-                "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
-                "traffic": profiled_traffic(args.workload), "ms_per_launch": round(t_assign, 5),
-                "algorithmic_flops_per_launch": flops}
+    if s.dtype == "f32":
+        # fp32 runs on the CUDA-core kernel: bound by the FP32 FMA pipes, whose
+        # peak is derived from the unit counts and the maximum SM clock
+        props = torch.cuda.get_device_properties(dev)
+        fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_GHZ / 1e3
+        roofline = {"bound": "alu", "kernel": "assign_simt_kernel", "achieved": round(tflops, 3),
+                    "peak": round(fp32_peak, 1), "unit": "TFLOP/s", "frac": round(tflops / fp32_peak, 4),
+                    "peak_kind": f"fp32 FMA: {props.multi_processor_count} SMs x {FP32_LANES_PER_SM} lanes x "
+                                 f"2 flop x {SM_MAX_GHZ} GHz (derived from unit counts and clock)",
+                    "traffic": None, "ms_per_launch": round(t_assign, 5), "algorithmic_flops_per_launch": flops}
+    else:
+        roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": round(tflops, 2),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(tflops / peaks["bf16_tflops"], 4),
+                    "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
+                    "traffic": profiled_traffic(args.workload), "ms_per_launch": round(t_assign, 5),
+                    "algorithmic_flops_per_launch": flops}
     roofline_update = {"bound": "hbm", "kernels": "fk_update (sort, offsets, segsum, finalize)",
                        "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peak_kind} copy",
