@@ -20,7 +20,9 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
                                                                 int D, int K,
                                                                 int32_t *__restrict__ labels,
                                                                 float *__restrict__ mindist) {
-  __shared__ float cs[kSimtTileK][DCH + 1];
+  // every lane reads the same centroid value (a broadcast), so rows need no
+  // padding, and 16-byte rows let a lane read four dimensions at once
+  __shared__ __align__(16) float cs[kSimtTileK][DCH];
   const int b = blockIdx.y;
   const int row = blockIdx.x * kSimtRows + threadIdx.x;
   const bool valid = row < N;
@@ -44,13 +46,18 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
       float xv[DCH];
 #pragma unroll
       for (int dd = 0; dd < DCH; ++dd) xv[dd] = (valid && d0 + dd < D) ? to_f32<T>(xrow[d0 + dd]) : 0.f;
-#pragma unroll 4
+      // fully unrolled, so that acc[] stays in registers
+#pragma unroll
       for (int t = 0; t < kSimtTileK; ++t) {
         float a = acc[t];
 #pragma unroll
-        for (int dd = 0; dd < DCH; ++dd) {
-          const float u = xv[dd] - cs[t][dd];
-          a = fmaf(u, u, a);
+        for (int dd = 0; dd < DCH; dd += 4) {
+          const float4 c4 = *reinterpret_cast<const float4 *>(&cs[t][dd]);
+          const float u0 = xv[dd] - c4.x, u1 = xv[dd + 1] - c4.y, u2 = xv[dd + 2] - c4.z, u3 = xv[dd + 3] - c4.w;
+          a = fmaf(u0, u0, a);
+          a = fmaf(u1, u1, a);
+          a = fmaf(u2, u2, a);
+          a = fmaf(u3, u3, a);
         }
         acc[t] = a;
       }
