@@ -231,6 +231,8 @@ def bench_gpu(args):
     B, N, D, K = s.B, s.N, s.D, s.K
     C = w.C0.clone()
     C_dt, bias = fk.fk_prepare_centroids(C, dt)
+    # |x|^2 of every point, once: X does not change between iterations
+    xnorm = fk.fk_prepare_points(X) if dt != torch.float32 else None
     labels = torch.empty(((B, N) if B > 1 else (N,)), dtype=torch.int32, device=dev)
     counts = torch.empty(((B, K) if B > 1 else (K,)), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -239,7 +241,7 @@ def bench_gpu(args):
         fk.fk_prepare_centroids(C, dt, C_dt, bias)
         if ev:
             ev[0].record(stream)
-        fk.fk_assign_prepared(X, C_dt, bias, labels)
+        fk.fk_assign_prepared(X, C_dt, bias, labels, xnorm=xnorm)
         if ev:
             ev[1].record(stream)
         fk.fk_update(X, labels, C, counts)

@@ -56,7 +56,8 @@ def _load():
         "fk_lloyd_ooc": [V, I64, I, I, V, I, V, V, I, I64, V],
         "fk_bias_len": [I, I],
         "fk_prepare_centroids": [V, I, I, I, I, V, V, V],
-        "fk_assign_prepared": [V, I, I64, I, I, V, I, V, V, V, V],
+        "fk_prepare_points": [V, I, I64, I, I, V, V],
+        "fk_assign_prepared": [V, I, I64, I, I, V, I, V, V, V, V, V],
         "fk_sync": [V],
         "fk_status_string": [I],
         "fk_get_last_error": [],
@@ -83,7 +84,7 @@ def _load():
 lib = _load()
 
 # names declared in include/fk.h (the C ABI this binding mirrors)
-ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
+ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_version")
@@ -166,12 +167,25 @@ def fk_prepare_centroids(C, dtype, C_dt=None, bias=None, stream=None):
     return C_dt, bias
 
 
-def fk_assign_prepared(X, C_dt, bias, labels, mindist=None, stream=None):
-    """One-kernel assignment against the output of ``fk_prepare_centroids``."""
+def fk_prepare_points(X, xnorm=None, stream=None):
+    """Row norms |x|^2 (fp32) of X (N x D or B x N x D), for fk_assign_prepared."""
+    B, N, D, bat = _dims(X)
+    lead = (B, N) if bat else (N,)
+    if xnorm is None:
+        xnorm = torch.empty(lead, dtype=torch.float32, device=X.device)
+    _need(xnorm, "xnorm", torch.float32, lead, X.device)
+    _check(lib.fk_prepare_points(_ptr(X), B, N, D, _dtype(X), _ptr(xnorm), _stream(stream)))
+    return xnorm
+
+
+def fk_assign_prepared(X, C_dt, bias, labels, mindist=None, xnorm=None, stream=None):
+    """Assignment against the output of ``fk_prepare_centroids`` (and
+    optionally of ``fk_prepare_points``): the assignment kernel and the exact
+    re-decision of near-ties."""
     B, N, D, bat = _dims(X)
     K = C_dt.shape[-2]
-    _check(lib.fk_assign_prepared(_ptr(X), B, N, D, _dtype(X), _ptr(C_dt), K, _ptr(bias), _ptr(labels),
-                                  _ptr(mindist), _stream(stream)))
+    _check(lib.fk_assign_prepared(_ptr(X), B, N, D, _dtype(X), _ptr(C_dt), K, _ptr(bias), _ptr(xnorm),
+                                  _ptr(labels), _ptr(mindist), _stream(stream)))
     return labels, mindist
 
 

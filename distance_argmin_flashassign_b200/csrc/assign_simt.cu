@@ -6,7 +6,13 @@
 // the centroids through shared memory in tiles of 32, keeps the 32 partial
 // squared distances in registers and folds them into a running (min, argmin)
 // in ascending centroid order, so ties go to the lowest index.  The distance
-// is the direct difference sum_j (x_j - c_j)^2 in fp32.
+// is the direct difference sum_j (x_j - c_j)^2 in fp32.  Per tile of 32
+// centroids (a chunk) the runner-up is tracked too: the smallest distance of
+// the other chunks and its chunk, the second smallest of the other chunks,
+// and the second smallest within the best chunk.  A point whose best and
+// runner-up distances lie within the fp32 rounding bound of each other is
+// listed for the exact re-decision (refine.cu) with the runner-up chunk, or
+// with -2 (every chunk) when a third chunk is that close too.
 #include "fk_internal.h"
 
 namespace fk {
@@ -19,7 +25,8 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
                                                                 const T *__restrict__ C, int N,
                                                                 int D, int K,
                                                                 int32_t *__restrict__ labels,
-                                                                float *__restrict__ mindist) {
+                                                                float *__restrict__ mindist,
+                                                                NearTies ties) {
   // every lane reads the same centroid value (a broadcast), so rows need no
   // padding, and 16-byte rows let a lane read four dimensions at once
   __shared__ __align__(16) float cs[kSimtTileK][DCH];
@@ -29,8 +36,9 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
   const T *xrow = X + ((size_t)b * N + (valid ? row : 0)) * D;
   const T *Cb = C + (size_t)b * K * D;
 
-  float best = __int_as_float(0x7f800000);
-  int bidx = 0;
+  const float inf = __int_as_float(0x7f800000);
+  float best = inf, s2 = inf, s3 = inf, s2in = inf;
+  int bidx = 0, bbase = 0, base2 = -1;
   for (int k0 = 0; k0 < K; k0 += kSimtTileK) {
     float acc[kSimtTileK];
 #pragma unroll
@@ -62,40 +70,67 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
         acc[t] = a;
       }
     }
+    // the chunk's smallest and second smallest distance, in centroid order
+    float m = inf, m2 = inf;
+    int mi = 0;
 #pragma unroll
     for (int t = 0; t < kSimtTileK; ++t) {
-      if (k0 + t < K && acc[t] < best) {
-        best = acc[t];
-        bidx = k0 + t;
+      const float a = k0 + t < K ? acc[t] : inf;
+      if (a < m) {
+        m2 = m;
+        m = a;
+        mi = t;
+      } else if (a < m2) {
+        m2 = a;
       }
     }
+    const bool imp = m < best;  // strict: an earlier chunk keeps a tie
+    const float lo = fmaxf(m, best);
+    const int lob = imp ? bbase : k0;
+    s3 = fminf(s3, fmaxf(lo, s2));
+    const bool up = lo < s2;
+    s2 = up ? lo : s2;
+    base2 = up ? lob : base2;
+    if (imp) {
+      best = m;
+      bidx = k0 + mi;
+      bbase = k0;
+      s2in = m2;
+    }
   }
+  const size_t g = (size_t)b * N + row;
   if (valid) {
-    labels[(size_t)b * N + row] = bidx;
-    if (mindist) mindist[(size_t)b * N + row] = best;
+    labels[g] = bidx;
+    if (mindist) mindist[g] = best;
+  }
+  if (ties.list != nullptr) {
+    const float second = fminf(s2, s2in);
+    const bool near = valid && second < inf && (second - best) <= ties.tau * (best + second);
+    const bool full = s3 < inf && (s3 - best) <= ties.tau * (best + s3);
+    list_append(ties, near, full, (int)g, base2);
   }
 }
 
 template <typename T>
 static cudaError_t launch_t(const void *X, const void *C, int B, int N, int D, int K, int32_t *labels,
-                            float *mindist, cudaStream_t s) {
+                            float *mindist, NearTies ties, cudaStream_t s) {
   dim3 grid((N + kSimtRows - 1) / kSimtRows, B);
   if (D <= 32)
     assign_simt_kernel<T, 32><<<grid, kSimtRows, 0, s>>>((const T *)X, (const T *)C, N, D, K, labels,
-                                                         mindist);
+                                                         mindist, ties);
   else
     assign_simt_kernel<T, 64><<<grid, kSimtRows, 0, s>>>((const T *)X, (const T *)C, N, D, K, labels,
-                                                         mindist);
+                                                         mindist, ties);
   count_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
-                               int32_t *labels, float *mindist, cudaStream_t s) {
+                               int32_t *labels, float *mindist, NearTies ties, cudaStream_t s) {
   switch (dt) {
-    case kF32: return launch_t<float>(X, C, B, N, D, K, labels, mindist, s);
-    case kF16: return launch_t<__half>(X, C, B, N, D, K, labels, mindist, s);
-    default: return launch_t<__nv_bfloat16>(X, C, B, N, D, K, labels, mindist, s);
+    case kF32: return launch_t<float>(X, C, B, N, D, K, labels, mindist, ties, s);
+    case kF16: return launch_t<__half>(X, C, B, N, D, K, labels, mindist, ties, s);
+    default: return launch_t<__nv_bfloat16>(X, C, B, N, D, K, labels, mindist, ties, s);
   }
 }
 

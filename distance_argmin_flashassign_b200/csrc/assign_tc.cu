@@ -94,10 +94,10 @@ template <int KB, bool DX> struct TcCfg {
   static constexpr int NSLOT = DX ? (KB == 1 ? 4 : 2) : (KB == 1 ? 9 : 4);  // tile slots in the ring
   static constexpr int X_BYTES = XBUF * KB * kXBytes;
   static constexpr int C_BYTES = NSLOT * SLOT;
-  static constexpr int XCHG_BYTES = kRows * 16;    // one float4 per row
+  static constexpr int XCHG_BYTES = kRows * 32;    // two float4 per row
   // full/empty per slot, xfull/xempty per X buffer, accfull/accempty per
-  // accumulator, xchg full/empty, drain
-  static constexpr int NBAR = 2 * NSLOT + 2 * XBUF + 2 * kAcc + 2 + 1;
+  // accumulator, xchg full/empty, drain, xready per X buffer
+  static constexpr int NBAR = 2 * NSLOT + 2 * XBUF + 2 * kAcc + 2 + 1 + XBUF;
   static constexpr int USED = X_BYTES + C_BYTES + XCHG_BYTES + kOnesBytes + NBAR * 8 + 16;
   static_assert(SLOT % 1024 == 0, "slots keep the 1 KB alignment of the 128-byte swizzle");
   static_assert(USED + 1024 <= 232448, "shared memory (227 KB per CTA on sm_100) exceeded");
@@ -165,15 +165,32 @@ struct TcParams {
   uint32_t dyn_bytes;
   int32_t *labels;
   float *mindist;
+  const float *xnorm;  // |x|^2 per row (B*N), or null: computed from the X tile
+  NearTies ties;  // where points whose two best scores are too close to order are listed
   DevCtl ctl;
 };
 
-// Running arg-max of one point over the chunks it has seen, in column order.
+// Running arg-max of one point over the chunks it has seen, in column order,
+// and the two best maxima of the other chunks (the runner-up chunk's, with
+// its first column, and the third chunk's).
 struct Best {
   float score;
   int base;           // first column of the candidate chunk
+  float s2;           // largest chunk maximum among the other chunks
+  int base2;          // first column of the chunk holding s2 (-1: none yet)
+  float s3;           // second largest chunk maximum among the other chunks
   uint32_t cand[32];  // the chunk that first reached `score`
 };
+
+__device__ __forceinline__ void best_init(Best &bs) {
+  bs.score = __int_as_float(0xff800000);
+  bs.base = 0;
+  bs.s2 = __int_as_float(0xff800000);
+  bs.base2 = -1;
+  bs.s3 = __int_as_float(0xff800000);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
+}
 
 // (d0, d1) = (a0 + b0, a1 + b1) in one packed fp32 add (FMA pipe).
 __device__ __forceinline__ void add2(uint32_t &d0, uint32_t &d1, uint32_t a0, uint32_t a1, uint32_t b0,
@@ -184,14 +201,33 @@ __device__ __forceinline__ void add2(uint32_t &d0, uint32_t &d1, uint32_t a0, ui
       : "r"(a0), "r"(a1), "r"(b0), "r"(b1));
 }
 
+// (a0, a1) += (v0 * v0, v1 * v1) in one packed fp32 fma.
+__device__ __forceinline__ void fma2(uint32_t &a0, uint32_t &a1, uint32_t v0, uint32_t v1) {
+  asm("{\n\t.reg .b64 a, v;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 v, {%2, %3};\n\t"
+      "fma.rn.f32x2 a, v, v, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+r"(a0), "+r"(a1)
+      : "r"(v0), "r"(v1));
+}
+
 // Fold one 32-column chunk of scores (first column `col`) into the running
 // arg-max.  The candidate copy is written as x + 0 (packed add.rn.f32x2, two
 // values per instruction on the FMA pipe, leaving the half-rate logic pipe
 // to the max trees); it keeps every value but turns -0 into +0, which
 // compares equal, so the index search below finds the same column.
+//
+// The chunk that does not hold the running maximum after the fold (the new
+// chunk, or the previous holder when the new chunk beats it) competes for
+// the runner-up chunk: its maximum min(m, score) replaces s2 when larger,
+// and the smaller of the two competes for s3.
 __device__ __forceinline__ void fold_chunk(Best &bs, const uint32_t (&v)[32], int col) {
   const float m = max32(v);
   const bool imp = m > bs.score;  // strict: an earlier column keeps a tie
+  const float lo = fminf(m, bs.score);
+  const int lob = imp ? bs.base : col;
+  bs.s3 = fmaxf(bs.s3, fminf(lo, bs.s2));
+  const bool up = lo > bs.s2;
+  bs.s2 = up ? lo : bs.s2;
+  bs.base2 = up ? lob : bs.base2;
   if (__any_sync(0xffffffffu, imp)) {
     if (imp) {
 #pragma unroll
@@ -200,6 +236,35 @@ __device__ __forceinline__ void fold_chunk(Best &bs, const uint32_t (&v)[32], in
       bs.base = col;
     }
   }
+}
+
+// Largest score of the candidate chunk other than the one at position jm.
+__device__ __forceinline__ float second_in_chunk(const Best &bs, int jm) {
+  float m[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) m[c] = __int_as_float(0xff800000);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float v = i == jm ? __int_as_float(0xff800000) : __uint_as_float(bs.cand[i]);
+    m[i & 3] = fmaxf(m[i & 3], v);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// A point whose best score s1 and runner-up s2 differ by no more than the
+// fp32 rounding of the scores may be ordered wrongly: it is listed for the
+// exact re-decision (refine.cu) together with the first column of the other
+// chunk it must re-examine, or for a comparison with every centroid when
+// the best maximum of a third chunk, s3, is that close too.  |x|^2 + |c_best|^2 <= 5|x|^2 - 4 s1
+// (as |c| <= |x| + |x - c| and |x - c|^2 = |x|^2 - 2 s1) bounds the
+// magnitudes the scores are accumulated from.  The warp appends its listed
+// points with one atomic add.
+__device__ __forceinline__ void list_near_tie(const NearTies &t, bool valid, float s1, float s2, float s3,
+                                              float xn, size_t g, int other) {
+  if (t.list == nullptr) return;
+  const float thr = t.tau * fmaxf(5.f * xn - 4.f * s1, 0.f);
+  const bool near = valid && (s1 - s2) <= thr;
+  list_append(t, near, (s1 - s3) <= thr, (int)g, other);
 }
 
 template <int KB, bool DX>
@@ -249,6 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t xchg_full = bar0 + 8u * (2 * NST + 2 * XBUF + 2 * kAcc);
   const uint32_t xchg_empty = xchg_full + 8u;
   const uint32_t drain = xchg_full + 16u;
+  // (one tile per unit) the peer's X tile has landed: the leader's epilogue
+  // sees the pair's xfull and tells the peer
+  auto xready = [&](int x) { return drain + 8u + 8u * x; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -259,6 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < XBUF; ++x) {
       mbar_init(xfull(x), 1);
       mbar_init(xempty(x), p.ntiles == 1 ? kEpiWarps / 2 : kEpiWarps);  // this CTA's warps of the unit, after it
+      mbar_init(xready(x), 1);  // one leader warp of the unit (read in the peer, one tile per unit)
     }
     // With one tile per unit each unit is read by one warp of each lane
     // quarter (see the epilogue), else by all epilogue warps.
@@ -411,8 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) mbar_arrive(accempty(a));
       else mbar_arrive_cluster_relaxed(map_to_cta(accempty(a), 0));
     };
-    // lowest column of the candidate chunk holding the maximum
-    auto best_index = [&](const Best &bs) {
+    // position (0-31) of the lowest column of the candidate chunk holding the
+    // maximum, 32 if none does
+    auto best_pos = [&](const Best &bs) {
       int j0 = 32, j1 = 32, j2 = 32, j3 = 32;
 #pragma unroll
       for (int i = 28; i >= 0; i -= 4) {
@@ -421,37 +491,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         j2 = __uint_as_float(bs.cand[i + 2]) == bs.score ? i + 2 : j2;
         j3 = __uint_as_float(bs.cand[i + 3]) == bs.score ? i + 3 : j3;
       }
-      const int jm = min(min(j0, j1), min(j2, j3));
-      return jm < 32 ? bs.base + jm : 0;
+      return min(min(j0, j1), min(j2, j3));
     };
-    // |x|^2 of this thread's row from the swizzled X tile in buffer xb: every
-    // MMA of the unit is done (its last accumulator was full), so X is
-    // resident until this CTA's warps of the unit have arrived on xempty
-    auto x_norm = [&](uint32_t xb) {
-      float xn = 0.f;
-      for (int kb = 0; kb < KB; ++kb) {
+    // Partial |x|^2 of this thread's row over its 16-byte groups [g0, g1) (8
+    // per k-block) from the swizzled X tile in buffer xb, which must have
+    // landed (it stays resident until this CTA's warps of the unit have
+    // arrived on xempty).  Squares of fp16/bf16 values are exact in fp32; the
+    // sums run two at a time (packed fma).
+    auto x_norm = [&](uint32_t xb, int g0, int g1) {
+      uint32_t a0 = 0u, a1 = 0u;
+      for (int gi = g0; gi < g1; ++gi) {
+        const int kb = gi >> 3, c = gi & 7;
         const uint8_t *rowp = sm + (xb * KB + kb) * kXBytes + r * 128;
+        const uint4 wv = *reinterpret_cast<const uint4 *>(rowp + ((c ^ (r & 7)) << 4));
+        const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 wv = *reinterpret_cast<const uint4 *>(rowp + ((c ^ (r & 7)) << 4));
-          const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float lo, hi;
-            if (p.is_bf16) {
-              lo = __uint_as_float(ws[e] << 16);
-              hi = __uint_as_float(ws[e] & 0xffff0000u);
-            } else {
-              const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[e]);
-              lo = __low2float(h2);
-              hi = __high2float(h2);
-            }
-            xn = fmaf(lo, lo, xn);
-            xn = fmaf(hi, hi, xn);
+        for (int e = 0; e < 4; ++e) {
+          uint32_t lo, hi;
+          if (p.is_bf16) {
+            lo = ws[e] << 16;
+            hi = ws[e] & 0xffff0000u;
+          } else {
+            const __half2 h2 = *reinterpret_cast<const __half2 *>(&ws[e]);
+            lo = __float_as_uint(__low2float(h2));
+            hi = __float_as_uint(__high2float(h2));
           }
+          fma2(a0, a1, lo, hi);
         }
       }
-      return xn;
+      return __uint_as_float(a0) + __uint_as_float(a1);
     };
     // The accumulators start out free.
     tc_fence_before();
@@ -473,10 +541,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
         const uint32_t xb = (uint32_t)(t % XBUF);
         Best bs;
-        bs.score = __int_as_float(0xff800000);
-        bs.base = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
+        best_init(bs);
+        // |x|^2 of this thread's row while the unit is multiplied: the X tile
+        // has landed once the pair's xfull completes (the leader sees it and
+        // tells the peer)
+        // (or read the prepared |x|^2, a load issued before the unit's wait)
+        float xn;
+        if (p.xnorm) {
+          xn = row < p.N ? __ldg(p.xnorm + (size_t)b * p.N + row) : 0.f;
+        } else {
+          const uint32_t xph = (uint32_t)(t / XBUF) & 1u;
+          if (leader) {
+            if (!(ok = mbar_wait(xfull(xb), xph, abort_flag, p.ctl))) break;
+            if (q == 0 && lane == 0) mbar_arrive_cluster(map_to_cta(xready(xb), 1));
+          } else {
+            if (!(ok = mbar_wait_acq_cluster(xready(xb), xph, abort_flag, p.ctl))) break;
+          }
+          xn = x_norm(xb, 0, KB * 8);
+        }
         if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
         tc_fence_after();
         if (q == 0 && lane == 0) mbar_arrive(empty(t % NST));  // the MMA is done with the slot
@@ -510,12 +592,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) release_acc(a);
         fold_chunk(bs, va, 192);
         fold_chunk(bs, vb, 224);
-        const int bi = best_index(bs);
+        const int jm = best_pos(bs);
+        const int bi = jm < 32 ? bs.base + jm : 0;
+        const float s2 = fmaxf(bs.s2, second_in_chunk(bs, jm));
+        const size_t o_ = (size_t)b * p.N + row;
         if (row < p.N) {
-          const size_t o_ = (size_t)b * p.N + row;
           p.labels[o_] = bi;
-          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, bs.score, x_norm(xb)));
+          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, bs.score, xn));
         }
+        list_near_tie(p.ties, row < p.N, bs.score, s2, bs.s3, xn, o_, bs.base2);
         __syncwarp();
         if (lane == 0) mbar_arrive(xempty(xb));
       }
@@ -527,10 +612,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = u / p.upb;
         const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
         Best bs;
-        bs.score = __int_as_float(0xff800000);
-        bs.base = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) bs.cand[i] = 0u;
+        best_init(bs);
+        // this column half's share of |x|^2, or (column half 0) the prepared
+        // |x|^2, loaded now and used at the end of the unit
+        float xn = 0.f;
+        if (p.xnorm && h == 0 && row < p.N) xn = __ldg(p.xnorm + (size_t)b * p.N + row);
         for (int j = 0; ok && j < p.ntiles; ++j, ++t) {
           const int a = t & 1;
           if (!(ok = mbar_wait(accfull(a), (uint32_t)(t >> 1) & 1u, abort_flag, p.ctl))) break;
@@ -557,15 +643,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) release_acc(a);
           fold_chunk(bs, vc, col + 64);
           fold_chunk(bs, va, col + 96);
+          // half of the row's |x|^2 per column half, while the unit's second
+          // tile is multiplied (the first tile's MMAs have read X)
+          if (j == 0 && !p.xnorm) xn = x_norm(xb, h * KB * 4, (h + 1) * KB * 4);
         }
         if (!ok) break;
-        const int bi = best_index(bs);
+        const int jm = best_pos(bs);
+        const int bi = jm < 32 ? bs.base + jm : 0;
+        const float s2in = second_in_chunk(bs, jm);
         // merge the two column halves of each point: half 1 hands over its
         // candidate and |x|^2, half 0 merges and writes
         if (h == 1) {
           if (u != u_begin && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
-          const float xn = p.mindist ? x_norm(xb) : 0.f;
-          xchg[r] = make_float4(bs.score, __int_as_float(bi), xn, 0.f);
+          xchg[2 * r] = make_float4(bs.score, __int_as_float(bi), xn, bs.s2);
+          xchg[2 * r + 1] = make_float4(s2in, __int_as_float(bs.base2), bs.s3, 0.f);
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(xchg_full);
@@ -573,16 +664,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           if (!(ok = mbar_wait(xchg_full, xc, abort_flag, p.ctl))) break;
-          const float4 o = xchg[r];
-          float sb = bs.score;
-          int bb = bi;
-          const int oi = __float_as_int(o.y);
-          if (o.x > sb || (o.x == sb && oi < bb)) { sb = o.x; bb = oi; }
+          const float4 o = xchg[2 * r], o2 = xchg[2 * r + 1];
+          const float xt = xn + o.z;
+          const int oi = __float_as_int(o.y), ob2 = __float_as_int(o2.y);
+          // winner: larger score, then lower column; runner-up chunk: the
+          // better of the loser's best chunk and the winner's own runner-up
+          const bool other_wins = o.x > bs.score || (o.x == bs.score && oi < bi);
+          const float s1 = other_wins ? o.x : bs.score;
+          const int b1 = other_wins ? oi : bi;
+          const float w_s2 = other_wins ? o.w : bs.s2, w_in = other_wins ? o2.x : s2in;
+          const int w_b2 = other_wins ? ob2 : bs.base2;
+          const float l_s1 = other_wins ? bs.score : o.x;
+          const int l_b1 = other_wins ? bi : oi;
+          const float s2 = fmaxf(fmaxf(w_s2, w_in), l_s1);
+          const int other = l_s1 > w_s2 ? (l_b1 & ~31) : w_b2;
+          // third best among the other chunks: the winner's runner-up and third,
+          // the loser's best chunk and runner-up
+          const float w_s3 = other_wins ? o2.z : bs.s3, l_s2 = other_wins ? bs.s2 : o.w;
+          const float s3 = l_s1 >= w_s2 ? fmaxf(w_s2, l_s2) : fmaxf(l_s1, w_s3);
+          const size_t o_ = (size_t)b * p.N + row;
           if (row < p.N) {
-            const size_t o_ = (size_t)b * p.N + row;
-            p.labels[o_] = bb;
-            if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, sb, o.z));
+            p.labels[o_] = b1;
+            if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, s1, xt));
           }
+          list_near_tie(p.ties, row < p.N, s1, s2, s3, xt, o_, other);
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(xchg_empty);
@@ -697,8 +802,8 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
 }
 
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
-                             int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
-                             int num_sms, cudaStream_t s) {
+                             int D, int K, int Kpad, const float *xnorm, int32_t *labels, float *mindist,
+                             NearTies ties, DevCtl ctl, int num_sms, cudaStream_t s) {
   if (!tc_shape_ok(dt, D) || !tc_aligned(X, C) || (uintptr_t)bias % 16 != 0) return cudaErrorNotSupported;
   CUtensorMap xm, cm, bm;
   if (!encode_3d(&xm, dt, X, D, N, B, kRows) || !encode_3d(&cm, dt, C, D, K, B, kHalfN) ||
@@ -716,6 +821,8 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   p.is_bf16 = dt == kBF16;
   p.labels = labels;
   p.mindist = mindist;
+  p.xnorm = xnorm;
+  p.ties = ties;
   p.ctl = ctl;
   p.dyn_bytes = 0;
   if (p.total_units == 0) return cudaSuccess;

@@ -40,6 +40,9 @@ static fk_status cuda_fail(cudaError_t e, const char *where) {
 struct Scratch {
   void *ptr = nullptr;
   size_t bytes = 0;
+  // near-tie list counters of the assignment kernels (count, done), zeroed
+  // once on allocation; the re-decision kernel leaves them zero
+  int *ties_ctl = nullptr;
   // out-of-core driver: side copy stream and ring events, created on first use
   cudaStream_t copy = nullptr;
   cudaEvent_t ready[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
@@ -116,6 +119,37 @@ static fk_status ooc_streams(DevState &d, cudaStream_t s, Scratch **out) {
 
 static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
 
+// Bytes of scratch the near-tie list of an assignment of `rows` points takes.
+static size_t ties_bytes(int64_t rows) { return al256((size_t)rows * sizeof(int2)); }
+
+// The near-tie list of an assignment on (device, stream): `list` is scratch
+// of ties_bytes(rows); the counters are allocated (and zeroed) on first use.
+static fk_status near_ties(DevState &d, cudaStream_t s, void *list, int64_t rows, int D, NearTies *out) {
+  int *ctl = nullptr;
+  {
+    std::lock_guard<std::mutex> g(d.mu);
+    Scratch &w = d.scratch[s];
+    if (!w.ties_ctl) {
+      cudaError_t e = cudaMallocAsync((void **)&w.ties_ctl, 256, s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(w.ties_ctl, 0, 256, s);
+      if (e != cudaSuccess) {
+        if (w.ties_ctl) cudaFreeAsync(w.ties_ctl, s);
+        w.ties_ctl = nullptr;
+        cudaGetLastError();
+        return cuda_fail(e, "cudaMallocAsync(near-tie counters)");
+      }
+    }
+    ctl = w.ties_ctl;
+  }
+  out->list = (int2 *)list;
+  out->cap = (int)rows;
+  out->count = ctl;
+  out->done = ctl + 1;
+  out->count_hi = ctl + 2;
+  out->tau = near_tie_tau_simt(D);
+  return FK_OK;
+}
+
 static bool valid_dtype(fk_dtype dt) { return dt == FK_F32 || dt == FK_F16 || dt == FK_BF16; }
 
 static fk_status check_sizes(int B, int64_t N, int D, int K, fk_dtype dt) {
@@ -139,12 +173,19 @@ static int choose_path(DType dt, int D) {
 
 // Assignment of B problems.  cn (the prepared bias of C: kBiasTerms floats per
 // padded centroid) may be null, in which case the tensor path computes it into
-// scratch at `cn_ws`.
+// scratch at `cn_ws`.  `ties_ws` is scratch of ties_bytes(B * N) for the
+// near-tie list; the points listed there are re-decided exactly (refine.cu)
+// by a second kernel.  xnorm (|x|^2 per point) may be null: the tensor-core
+// kernel then computes it from its X tiles.
 static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
-                            const float *cn, float *cn_ws, int32_t *labels, float *mindist,
-                            cudaStream_t s) {
+                            const float *cn, float *cn_ws, void *ties_ws, const float *xnorm, int32_t *labels,
+                            float *mindist, cudaStream_t s) {
+  NearTies ties;
+  fk_status st = near_ties(d, s, ties_ws, (int64_t)B * N, D, &ties);
+  if (st != FK_OK) return st;
   const int path = choose_path(dt, D);
   if (path < 0) return fail(FK_ERR_UNSUPPORTED, "tensor-core path forced for an unsupported shape");
+  bool done = false;
   if (path == 1 && tc_aligned(X, C) && (!cn || (uintptr_t)cn % 16 == 0)) {
     const int Kpad = pad_k(K);
     if (!cn) {
@@ -152,16 +193,26 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
       if (e != cudaSuccess) return cuda_fail(e, "bias kernel");
       cn = cn_ws;
     }
-    cudaError_t e = launch_assign_tc(dt, X, C, cn, B, N, D, K, Kpad, labels, mindist, ctl_of(d), d.sms, s);
-    if (e == cudaSuccess) return FK_OK;
-    if (e != cudaErrorNotSupported) return cuda_fail(e, "tensor-core assign kernel");
-    cudaGetLastError();
-    if (g_assign_path.load() == 1) return fail(FK_ERR_UNSUPPORTED, "tensor maps could not be encoded");
+    NearTies tt = ties;
+    tt.tau = kNearTieTauTc;
+    cudaError_t e =
+        launch_assign_tc(dt, X, C, cn, B, N, D, K, Kpad, xnorm, labels, mindist, tt, ctl_of(d), d.sms, s);
+    if (e == cudaSuccess) {
+      done = true;
+    } else {
+      if (e != cudaErrorNotSupported) return cuda_fail(e, "tensor-core assign kernel");
+      cudaGetLastError();
+      if (g_assign_path.load() == 1) return fail(FK_ERR_UNSUPPORTED, "tensor maps could not be encoded");
+    }
   } else if (path == 1 && g_assign_path.load() == 1) {
     return fail(FK_ERR_UNSUPPORTED, "tensor-core path needs 16-byte aligned X, C and bias");
   }
-  cudaError_t e = launch_assign_simt(dt, X, C, B, N, D, K, labels, mindist, s);
-  if (e != cudaSuccess) return cuda_fail(e, "CUDA-core assign kernel");
+  if (!done) {
+    cudaError_t e = launch_assign_simt(dt, X, C, B, N, D, K, labels, mindist, ties, s);
+    if (e != cudaSuccess) return cuda_fail(e, "CUDA-core assign kernel");
+  }
+  cudaError_t e = launch_refine(dt, X, C, N, D, K, ties, labels, mindist, d.sms, s);
+  if (e != cudaSuccess) return cuda_fail(e, "near-tie re-decision kernel");
   return FK_OK;
 }
 
@@ -216,8 +267,10 @@ fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dtype dt,
   if ((st = device_state(&d)) != FK_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   void *ws = nullptr;
-  if ((st = scratch(*d, s, al256(bias_bytes(B, K)), &ws)) != FK_OK) return st;
-  return run_assign(*d, (DType)dt, X, B, (int)N, D, C, K, nullptr, (float *)ws, labels, mindist, s);
+  const size_t cnb = al256(bias_bytes(B, K));
+  if ((st = scratch(*d, s, cnb + ties_bytes((int64_t)B * N), &ws)) != FK_OK) return st;
+  return run_assign(*d, (DType)dt, X, B, (int)N, D, C, K, nullptr, (float *)ws, (char *)ws + cnb, nullptr, labels,
+                    mindist, s);
 }
 
 fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, int32_t *labels,
@@ -248,15 +301,32 @@ fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype d
   return FK_OK;
 }
 
+fk_status fk_prepare_points(const void *X, int B, int64_t N, int D, fk_dtype dt, float *xnorm,
+                            fk_stream_t stream) {
+  fk_status st = check_sizes(B, N, D, 1, dt);
+  if (st != FK_OK) return st;
+  if (N == 0) return FK_OK;
+  if (!X || !xnorm) return fail(FK_ERR_INVALID_ARG, "X and xnorm must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaError_t e = launch_point_norms((DType)dt, X, (long long)B * N, D, xnorm, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "point norm kernel");
+  return FK_OK;
+}
+
 fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt, int K,
-                             const float *bias, int32_t *labels, float *mindist, fk_stream_t stream) {
+                             const float *bias, const float *xnorm, int32_t *labels, float *mindist,
+                             fk_stream_t stream) {
   fk_status st = check_sizes(B, N, D, K, dt);
   if (st != FK_OK) return st;
   if (N == 0) return FK_OK;
   if (!X || !C_dt || !labels || !bias) return fail(FK_ERR_INVALID_ARG, "X, C_dt, bias and labels must not be NULL");
   DevState *d;
   if ((st = device_state(&d)) != FK_OK) return st;
-  return run_assign(*d, (DType)dt, X, B, (int)N, D, C_dt, K, bias, nullptr, labels, mindist, (cudaStream_t)stream);
+  cudaStream_t s = (cudaStream_t)stream;
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, ties_bytes((int64_t)B * N), &ws)) != FK_OK) return st;
+  return run_assign(*d, (DType)dt, X, B, (int)N, D, C_dt, K, bias, nullptr, ws, xnorm, labels, mindist, s);
 }
 
 fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t N, int D, fk_dtype dt,
@@ -315,10 +385,18 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   const size_t upd = al256(update_workspace_bytes((int64_t)B * N, (int64_t)B * K, D, B));
   const size_t cnb = al256(bias_bytes(B, K));
   const size_t cdb = t == kF32 ? 0 : al256((size_t)B * K * D * dtype_size(t));
+  const size_t tb = ties_bytes((int64_t)B * N);
+  const size_t xb = t == kF32 ? 0 : al256((size_t)B * N * 4);
   void *ws = nullptr;
-  if ((st = scratch(*d, s, upd + cnb + cdb, &ws)) != FK_OK) return st;
+  if ((st = scratch(*d, s, upd + cnb + cdb + tb + xb, &ws)) != FK_OK) return st;
   float *cn = (float *)((char *)ws + upd);
   void *Cdt = t == kF32 ? (void *)C : (void *)((char *)ws + upd + cnb);
+  void *tl = (char *)ws + upd + cnb + cdb;
+  float *xn = t == kF32 ? nullptr : (float *)((char *)ws + upd + cnb + cdb + tb);
+  if (xn) {  // |x|^2 once for all iterations (X does not change)
+    cudaError_t e = launch_point_norms(t, X, (long long)B * N, D, xn, s);
+    if (e != cudaSuccess) return cuda_fail(e, "point norm kernel");
+  }
 
   UpdateArgs a{};
   a.dt = t;
@@ -336,7 +414,8 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
       cudaError_t e = launch_round_bias(t, C, B, K, Kpad, D, Cdt, cn, s);
       if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
     }
-    st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, labels, it == iters - 1 ? mindist : nullptr, s);
+    st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, tl, xn, labels, it == iters - 1 ? mindist : nullptr,
+                    s);
     if (st != FK_OK) return st;
     cudaError_t e = launch_update(a, ws, upd, ctl_of(*d), d->sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "update kernels");
@@ -377,7 +456,8 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
   const size_t b_cn = al256(bias_bytes(1, K)), b_acc = al256((size_t)K * D * 8);
   const size_t b_cnt = al256((size_t)K * 8), b_counts = al256((size_t)K * 4);
   const size_t b_upd = al256(update_workspace_bytes(rows, K, D, 1));
-  const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd;
+  const size_t b_ties = ties_bytes(rows);
+  const size_t total = 2 * b_ring + 2 * b_lab + b_c32 + b_cdt + b_cn + b_acc + b_cnt + b_counts + b_upd + b_ties;
 
   Scratch *sc = nullptr;
   char *mem = nullptr;
@@ -407,6 +487,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
     double *acc = (double *)p; p += b_acc;
     long long *cnt = (long long *)p; p += b_cnt;
     int32_t *cnts = (int32_t *)p; p += b_counts;
+    void *tl = (void *)p; p += b_ties;
     void *upd = (void *)p;
 
     // Order the copy stream after everything already queued on `s` (the
@@ -440,7 +521,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
         FK_TRY(cudaEventRecord(ready[slot], cs), "cudaEventRecord", FK_ERR_CUDA);
         // compute stream: assign the chunk and accumulate its per-cluster sums
         FK_TRY(cudaStreamWaitEvent(s, ready[slot], 0), "cudaStreamWaitEvent", FK_ERR_CUDA);
-        rc = run_assign(*d, t, ring[slot], 1, nr, D, cdt, K, cn, nullptr, lab[slot], nullptr, s);
+        rc = run_assign(*d, t, ring[slot], 1, nr, D, cdt, K, cn, nullptr, tl, nullptr, lab[slot], nullptr, s);
         if (rc != FK_OK) goto done;
         if (it == iters - 1 && labels_host)
           FK_TRY(cudaMemcpyAsync(labels_host + r0, lab[slot], (size_t)nr * 4, cudaMemcpyDeviceToHost, s),
@@ -528,6 +609,7 @@ fk_status fk_release_workspace(void) {
   std::lock_guard<std::mutex> g(d->mu);
   for (auto &kv : d->scratch) {
     if (kv.second.ptr) cudaFreeAsync(kv.second.ptr, kv.first);
+    if (kv.second.ties_ctl) cudaFreeAsync(kv.second.ties_ctl, kv.first);
   }
   cudaError_t e = cudaDeviceSynchronize();
   for (auto &kv : d->scratch) {  // the out-of-core side streams are idle now

@@ -25,6 +25,44 @@ struct DevCtl {
   unsigned long long timeout_ns;
 };
 
+// Points the assignment kernels could not order with certainty: a point
+// whose best and second-best fp32 scores (or distances) lie within `tau`
+// times the magnitude they were accumulated from is listed as (global row
+// b*N + i, first column of the second 32-centroid chunk to re-examine, or
+// -1).  When a third chunk is that close too, the point is listed as
+// (row, -2), from the other end of the list, for a comparison with every
+// centroid.  The re-decision kernel (refine.cu) reads both parts, decides
+// them exactly and resets the counts to 0.
+struct NearTies {
+  int2 *list;     // room for `cap` entries (B*N: a point is listed at most once)
+  int *count;     // entries [0, *count), zero before the assignment kernel runs
+  int *done;      // blocks of the re-decision kernel that have finished
+  int *count_hi;  // entries [cap - *count_hi, cap), the full comparisons
+  int cap;
+  float tau;
+};
+
+// Append the listed points of a warp (every lane calls this, `near` and
+// `full` per lane): two-chunk points with one atomic add per warp from the
+// front, full-comparison points one by one from the back.
+__device__ __forceinline__ void list_append(const NearTies &t, bool near, bool full, int g, int other) {
+  const bool two = near && !full;
+  const unsigned fm = __ballot_sync(0xffffffffu, two);
+  const int lane = threadIdx.x & 31;
+  if (fm != 0u) {
+    const int lead = __ffs(fm) - 1;
+    int at = 0;
+    if (lane == lead) at = atomicAdd(t.count, __popc(fm));
+    at = __shfl_sync(0xffffffffu, at, lead);
+    const int slot = at + __popc(fm & ((1u << lane) - 1u));
+    if (two && slot < t.cap) t.list[slot] = make_int2(g, other);
+  }
+  if (near && full) {
+    const int slot = t.cap - 1 - atomicAdd(t.count_hi, 1);
+    if (slot >= 0) t.list[slot] = make_int2(g, -2);
+  }
+}
+
 __device__ __forceinline__ void record_status(int *status, int code) {
   atomicCAS(status, 0, code);  // first error wins
 }
@@ -108,6 +146,33 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   const uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > ctl.timeout_ns) {
+      *abort = 1;
+      record_status(ctl.status, kStTimeout);
+      return false;
+    }
+  }
+}
+
+// mbar_wait for a barrier whose phase is completed by a thread of the other
+// CTA of the pair with a cluster-scope release: the test acquires at cluster
+// scope, so what that thread could see is visible here afterwards.
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(sleep_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity, volatile int *abort,
+                                                      const DevCtl &ctl) {
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_acq_cluster(bar, parity, kWaitSleepNs)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > ctl.timeout_ns) {
       *abort = 1;

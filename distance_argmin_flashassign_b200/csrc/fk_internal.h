@@ -15,6 +15,7 @@ void count_launches(int n);
 // Set the calling thread's last error (fk_get_last_error / fk_last_error_message).
 int record_error(int status, const char *msg);
 
+constexpr int kMaxD = 1024;        // largest D the library accepts
 constexpr int kCentroidPad = 256;  // centroid tile of the tensor-core kernel
 inline int pad_k(int K) { return (K + kCentroidPad - 1) / kCentroidPad * kCentroidPad; }
 // Floats of prepared bias per (padded) centroid: three tf32-exact terms of
@@ -28,21 +29,39 @@ inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
 // bias[b*Kpad + j] = -|C[b][j]|^2 / 2 in fp32 for j < K, -inf for K <= j < Kpad.
 cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, float *bias,
                         cudaStream_t s);
+// xnorm[r] = |X[r]|^2 (fp32) for the `rows` rows of D elements of X.
+cudaError_t launch_point_norms(DType dt, const void *X, long long rows, int D, float *xnorm, cudaStream_t s);
 // Cdt = C32 rounded to dt (round-to-nearest-even) and bias of Cdt.
 cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
                               float *bias, cudaStream_t s);
 
+// Relative width of the near-tie test of the CUDA-core kernel for rows of D
+// dimensions: (D + 8) units of fp32 rounding, the classical bound on the
+// error of an fp32 sum of D + 8 terms (the squared differences), times the
+// magnitude summed (the two distances).
+inline float near_tie_tau_simt(int D) { return (float)(D + 8) * 5.9604644775390625e-8f; }
+// The same for the tensor-core kernel: 16 units of fp32 rounding (2^-20)
+// times a bound on |x|^2 + |c|^2.  Its accumulation order is the hardware's;
+// on the five workloads no point whose score gap exceeded 1.3e-7 (|x|^2 +
+// |c|^2) was misordered, eight times below this width.
+constexpr float kNearTieTauTc = 9.5367431640625e-7f;
+
 // ---- assign_simt.cu: CUDA-core assignment (any dtype, any D) --------------
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
-                               int32_t *labels, float *mindist, cudaStream_t s);
+                               int32_t *labels, float *mindist, NearTies ties, cudaStream_t s);
+
+// ---- refine.cu: exact re-decision of listed near-ties ---------------------
+cudaError_t launch_refine(DType dt, const void *X, const void *C, int N, int D, int K, NearTies t,
+                          int32_t *labels, float *mindist, int num_sms, cudaStream_t s);
 
 // ---- assign_tc.cu: tcgen05 assignment (fp16/bf16, D % 8 == 0, D <= 128) --
 bool tc_shape_ok(DType dt, int D);
 bool tc_aligned(const void *X, const void *C);
 // Returns cudaErrorNotSupported if the tensor maps could not be encoded.
+// xnorm: |x|^2 per row (B*N floats), or null (computed in the kernel).
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
-                             int D, int K, int Kpad, int32_t *labels, float *mindist, DevCtl ctl,
-                             int num_sms, cudaStream_t s);
+                             int D, int K, int Kpad, const float *xnorm, int32_t *labels, float *mindist,
+                             NearTies ties, DevCtl ctl, int num_sms, cudaStream_t s);
 
 // ---- update.cu: sort-inverse update ---------------------------------------
 enum UpdateMode : int { kMean = 0, kAccumulate = 1 };

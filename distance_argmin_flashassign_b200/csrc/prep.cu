@@ -90,6 +90,40 @@ __global__ void __launch_bounds__(256) round_bias_kernel(const float *__restrict
   }
 }
 
+// |x|^2 of every row of X (fp32 sums of the squares, which are exact for
+// fp16/bf16 inputs): the row norms of the assignment stage, for its near-tie
+// test and its squared distances.  One warp per row, 16-byte loads when rows
+// are 16-byte multiples.
+template <typename T>
+__global__ void __launch_bounds__(256) point_norms_kernel(const T *__restrict__ X, long long rows, int D,
+                                                          int vec, float *__restrict__ xnorm) {
+  const int lane = threadIdx.x & 31;
+  for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += (long long)gridDim.x * 8) {
+    const T *x = X + (size_t)r * D;
+    float s = 0.f;
+    if (vec) {
+      constexpr int E = 16 / sizeof(T);
+      const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+      for (int v = lane; v < D / E; v += 32) {
+        const uint4 w = __ldg(xv + v);
+        const T *e = reinterpret_cast<const T *>(&w);
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float f = to_f32<T>(e[i]);
+          s = fmaf(f, f, s);
+        }
+      }
+    } else {
+      for (int d = lane; d < D; d += 32) {
+        const float f = to_f32<T>(x[d]);
+        s = fmaf(f, f, s);
+      }
+    }
+    s = warp_sum(s);
+    if (lane == 0) xnorm[r] = s;
+  }
+}
+
 static int grid_for_rows(long long rows) {
   long long g = (rows + 7) / 8;
   return (int)(g < 4096 ? (g < 1 ? 1 : g) : 4096);
@@ -103,6 +137,19 @@ cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, 
     case kF16: bias_kernel<__half><<<g, 256, 0, s>>>((const __half *)C, B, K, Kpad, D, bias); break;
     default:
       bias_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)C, B, K, Kpad, D, bias);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_point_norms(DType dt, const void *X, long long rows, int D, float *xnorm, cudaStream_t s) {
+  const int g = grid_for_rows(rows);
+  const int vec = ((size_t)D * dtype_size(dt)) % 16 == 0 && (uintptr_t)X % 16 == 0;
+  switch (dt) {
+    case kF32: point_norms_kernel<float><<<g, 256, 0, s>>>((const float *)X, rows, D, vec, xnorm); break;
+    case kF16: point_norms_kernel<__half><<<g, 256, 0, s>>>((const __half *)X, rows, D, vec, xnorm); break;
+    default:
+      point_norms_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)X, rows, D, vec, xnorm);
   }
   count_launches(1);
   return cudaGetLastError();

@@ -29,6 +29,15 @@
  *              (the pages are silent on ties).  mindist[i] = that squared
  *              distance, clamped at 0.  The tensor path ranks by
  *              <x,c> - |c|^2/2 in fp32 (mindist = |x|^2 - 2 * best score).
+ *   Exactness  Every assignment ends with an exact re-decision of the
+ *              points whose best and second-best fp32 values lie within the
+ *              fp32 rounding width of each other: their distances to the
+ *              centroids of the two 32-centroid chunks holding those values
+ *              (or to every centroid, when a third chunk is as close) are
+ *              recomputed as sum_j (x_j - c_j)^2 in fp64, j ascending, and
+ *              the first minimum is taken; such a point's mindist is that
+ *              fp64 distance rounded to fp32.  The labels are then those of
+ *              the fp64 definition on the same (rounded) inputs.
  *   Update     C_k = mean of the points with label k, in fp32; a cluster
  *              that receives no point keeps its previous centroid and gets
  *              count 0 (the pages are silent on empty clusters).
@@ -103,6 +112,9 @@ FK_API fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const v
                     int32_t *labels, float *mindist, fk_stream_t stream);
 
 /* fk_assign_batched -- B independent assignment problems in one launch.
+ *   Flash-KMeans abstract (FlashAssign) applied per problem; the batch of
+ *   independent problems in one launch is this library's reading of the
+ *   batched online-clustering use the Flash-KMeans pages motivate.
  *   X B x N x D, C B x K x D, labels B x N, mindist B x N or NULL (device).
  *   Problem b compares rows of X[b] only with centroids of C[b]; labels are
  *   in [0, K) within each problem. */
@@ -127,16 +139,25 @@ FK_API fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dt
  *   C32 device B x K x D fp32; C_dt device B x K x D of dt; bias device
  *   fk_bias_len(B, K) floats, 16-byte aligned for the tensor-core path (a
  *   less aligned bias sends fk_assign_prepared to the CUDA-core kernel).
+ * fk_prepare_points -- the row norms of the assignment stage:
+ *   xnorm[i] = |x_i|^2 in fp32 for the B*N rows of X (device, B x N x D of
+ *   dt; xnorm device, B*N floats).  X does not change between Lloyd
+ *   iterations, so an iterating caller computes this once.  One kernel.
  * fk_assign_prepared -- fk_assign_batched against prepared centroids and
- *   bias; launches exactly one kernel (the CUDA-core kernel, which computes
- *   direct differences, does not read the bias).
+ *   bias, and optionally the prepared row norms (xnorm, or NULL: the
+ *   tensor-core kernel then sums them from its X tiles).  Launches two
+ *   kernels: the assignment kernel (the CUDA-core kernel, which computes
+ *   direct differences, reads neither the bias nor xnorm) and the exact
+ *   re-decision of near-ties (see "Exactness" below).
  * ------------------------------------------------------------------------ */
 FK_API int64_t fk_bias_len(int B, int K);
 FK_API fk_status fk_prepare_centroids(const float *C32, int B, int K, int D, fk_dtype dt, void *C_dt,
                                       float *bias, fk_stream_t stream);
+FK_API fk_status fk_prepare_points(const void *X, int B, int64_t N, int D, fk_dtype dt, float *xnorm,
+                                   fk_stream_t stream);
 FK_API fk_status fk_assign_prepared(const void *X, int B, int64_t N, int D, fk_dtype dt, const void *C_dt,
-                                    int K, const float *bias, int32_t *labels, float *mindist,
-                                    fk_stream_t stream);
+                                    int K, const float *bias, const float *xnorm, int32_t *labels,
+                                    float *mindist, fk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * fk_update -- centroid-update stage (sort-inverse update).
@@ -159,7 +180,9 @@ FK_API fk_status fk_update(const void *X, const int32_t *labels, int64_t N, int 
                     float *C, int32_t *counts, fk_stream_t stream);
 
 /* fk_update_batched -- B independent update problems (labels B x N, C B x K
- * x D fp32 in/out, counts B x K or NULL), one sort over B*K segments. */
+ * x D fp32 in/out, counts B x K or NULL), one sort over B*K segments.
+ * Flash-KMeans abstract (sort-inverse update) applied per problem, in one
+ * launch per kernel for the whole batch. */
 FK_API fk_status fk_update_batched(const void *X, const int32_t *labels, int B, int64_t N, int D,
                             fk_dtype dt, int K, float *C, int32_t *counts, fk_stream_t stream);
 
@@ -195,6 +218,9 @@ FK_API fk_status fk_update_noalloc(const void *X, const int32_t *labels, int64_t
 
 /* ------------------------------------------------------------------------
  * fk_lloyd -- `iters` Lloyd iterations, device resident.
+ *   Flash-KMeans abstract: one iteration is the assignment stage followed by
+ *   the centroid-update stage; the Japanese Hacker News summary, key points:
+ *   the k-means mathematics itself is unchanged.
  *   Iteration t assigns X against C_t rounded (round-to-nearest-even) to the
  *   input type (fp16/bf16; fp32 uses C_t as is), then sets C_{t+1} = the
  *   cluster means in fp32.  On return C holds C_iters, labels the last
@@ -208,7 +234,8 @@ FK_API fk_status fk_lloyd(const void *X, int64_t N, int D, fk_dtype dt, float *C
                    fk_stream_t stream);
 
 /* fk_lloyd_batched -- fk_lloyd over B independent problems in one launch per
- * stage (shapes as in fk_assign_batched / fk_update_batched). */
+ * stage (shapes as in fk_assign_batched / fk_update_batched); the iteration
+ * follows the Flash-KMeans abstract for each problem. */
 FK_API fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, float *C, int K,
                            int32_t *labels, float *mindist, int32_t *counts, int iters,
                            fk_stream_t stream);

@@ -33,8 +33,10 @@ _lib = None
 
 
 def build(src: str = _SRC, out: str = _LIB_PATH, openmp: bool = True) -> str:
-    """Compile the C oracle into a shared library (gcc, -O2, OpenMP)."""
-    cmd = ["gcc", "-O2", "-std=c11", "-shared", "-fPIC", src, "-o", out, "-lm"]
+    """Compile the C oracle into a shared library (gcc, -O2, OpenMP).  Every
+    multiply and add is rounded on its own: no contraction into fused
+    multiply-adds, which the plain definition does not perform."""
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-shared", "-fPIC", src, "-o", out, "-lm"]
     if openmp:
         cmd.insert(1, "-fopenmp")
     subprocess.run(cmd, check=True)

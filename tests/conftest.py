@@ -17,3 +17,19 @@ def pytest_configure(config):
 def oracle_lib():
     import oracle
     return oracle.load()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the parity statistics of every label comparison of the run."""
+    try:
+        from tests.parity import STATS
+    except Exception:
+        return
+    if not STATS:
+        return
+    tr = terminalreporter
+    tr.section("parity statistics (label comparisons against the oracle)")
+    keys = ["N", "mismatch", "near_tie_points", "fp32_ties", "centroid_rel_l2", "slack"]
+    for d in STATS:
+        tr.write_line(d["case"] + ": " + ", ".join(f"{k}={d[k]:.3g}" if isinstance(d.get(k), float)
+                                                   else f"{k}={d[k]}" for k in keys if k in d))

@@ -1,22 +1,23 @@
 """Comparison rules between the CUDA library and the CPU oracle.
 
-Acceptance (Flash-KMeans is exact k-means, arXiv 2603.09229 abstract; the
+Acceptance (Flash-KMeans is exact k-means: arXiv 2603.09229, abstract, and
+the Japanese Hacker News summary, results paragraph, "exact execution"; the
 tolerances are the project's stated bar):
 
 * labels are bit-exact, except at near-ties: a point may carry another label
   than the oracle's only if, in fp64, its distance to the GPU's centroid
   exceeds the minimum by at most ``band * (|x|^2 + |c_best|^2)`` with
   band = 1e-4 for fp32 inputs and 1e-2 for fp16/bf16 inputs (c_best is the
-  oracle's centroid); and such points are at most 0.01 % of N -- not counting
-  the points whose two distances the kernel's own fp32 arithmetic cannot
-  separate.  The argmin is decided in the kernel's precision (the pages fix
-  none): a mismatch whose fp64 distance excess is within the worst-case
-  rounding error of the fp32 evaluation, ``4 * gamma_D * (|x|^2 + |c|^2)``
-  with gamma_D = D u / (1 - D u), u = 2^-24 (the classical bound on an fp32
-  dot product of length D, applied to both candidates), is a valid answer
-  and is reported, not capped;
-* centroids within 1e-4 relative L2 (Frobenius) of the oracle's;
+  oracle's centroid); and EVERY such mismatch counts against the cap of
+  0.01 % of N (of the rows compared);
+* centroids within 1e-4 relative L2 (Frobenius) of the oracle's centroids,
+  which the oracle computes from its own labels;
 * counts (integers) exact.
+
+Each comparison's statistics (rows compared, mismatches, near-tie points,
+and, as a diagnostic only, how many mismatches lie within the worst-case
+rounding error of an fp32 evaluation) are appended to ``STATS`` and printed
+in the pytest terminal summary.
 """
 from __future__ import annotations
 
@@ -29,6 +30,14 @@ BAND = {"f32": 1e-4, "f16": 1e-2, "bf16": 1e-2}
 MINDIST_TOL = {"f32": 1e-5, "f16": 1e-3, "bf16": 1e-3}
 MAX_MISMATCH_FRAC = 1e-4
 CENTROID_REL_L2 = 1e-4
+
+STATS: list = []  # one dict per comparison, printed by tests/conftest.py
+
+
+def record(case: str, **stats) -> dict:
+    d = {"case": case, **stats}
+    STATS.append(d)
+    return d
 
 TORCH_DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
@@ -43,42 +52,45 @@ def f64(t: torch.Tensor) -> np.ndarray:
 
 def fp32_separation(D: int) -> float:
     """Relative width within which fp32 evaluation of |x|^2+|c|^2-2<x,c>
-    cannot order two centroids (times |x|^2 + |c|^2)."""
+    cannot order two centroids (times |x|^2 + |c|^2).  Diagnostic only: it
+    classifies mismatches in the reported statistics and exempts none."""
     u = 2.0 ** -24
     gamma = (D + 2) * u / (1 - (D + 2) * u)
     return 4.0 * gamma
 
 
 def check_labels(X64: np.ndarray, C64: np.ndarray, gpu_labels, dtype: str, gpu_mindist=None,
-                 exact: bool = False, max_frac: float = MAX_MISMATCH_FRAC):
+                 exact: bool = False, max_frac: float = MAX_MISMATCH_FRAC, case: str = ""):
     """Compare GPU labels (and mindist) with the oracle on the same rounded inputs.
 
-    Returns a dict of statistics; raises AssertionError when the bar is missed."""
+    Returns a dict of statistics (also recorded in ``STATS`` when ``case`` is
+    given); raises AssertionError when the bar is missed."""
     gl = np.asarray(gpu_labels.cpu() if torch.is_tensor(gpu_labels) else gpu_labels).astype(np.int64)
     lab, mind, second = oracle.assign(X64, C64)
     N = len(lab)
     assert gl.min(initial=0) >= 0 and gl.max(initial=0) < C64.shape[0], "label out of range"
     mism = np.nonzero(gl != lab)[0]
-    stats = {"N": N, "mismatch": int(len(mism)), "near_tie_points": 0}
     scale = (X64 ** 2).sum(1) + (C64[lab] ** 2).sum(1)
     gap = second - mind
-    stats["near_tie_points"] = int((gap <= BAND[dtype] * scale).sum())
-    if exact:
-        assert len(mism) == 0, f"{len(mism)} label mismatches where bit-exactness is required: {mism[:10]}"
+    stats = {"N": N, "mismatch": int(len(mism)),
+             "near_tie_points": int((gap <= BAND[dtype] * scale).sum()), "fp32_ties": 0}
     if len(mism):
         d_gpu = ((X64[mism] - C64[gl[mism]]) ** 2).sum(1)
         excess = d_gpu - mind[mism]
+        scale_gpu = (X64[mism] ** 2).sum(1) + (C64[gl[mism]] ** 2).sum(1)
+        stats["fp32_ties"] = int((excess <= fp32_separation(X64.shape[1]) *
+                                  np.maximum(scale[mism], scale_gpu)).sum())
+    if case:
+        stats = record(case, **stats)
+    if exact:
+        assert len(mism) == 0, f"{len(mism)} label mismatches where bit-exactness is required: {mism[:10]}"
+    if len(mism):
         bad = excess > BAND[dtype] * scale[mism]
         assert not bad.any(), (f"{int(bad.sum())} mismatches outside the near-tie band, e.g. row "
                                f"{mism[bad][0]}: excess {excess[bad][0]:.3g} vs band "
                                f"{BAND[dtype] * scale[mism][bad][0]:.3g}")
-        scale_gpu = (X64[mism] ** 2).sum(1) + (C64[gl[mism]] ** 2).sum(1)
-        rounding = excess <= fp32_separation(X64.shape[1]) * np.maximum(scale[mism], scale_gpu)
-        stats["fp32_ties"] = int(rounding.sum())
-        beyond = int((~rounding).sum())
-        stats["capped_mismatch"] = beyond
-        assert beyond <= max_frac * N, (f"{beyond} mismatches beyond fp32 rounding (of {len(mism)}) > "
-                                        f"{max_frac:.2%} of {N}")
+        assert len(mism) <= max_frac * N, (f"{len(mism)} label mismatches (near-ties) > "
+                                           f"{max_frac:.2%} of {N} rows")
     if gpu_mindist is not None:
         gm = np.asarray(gpu_mindist.cpu() if torch.is_tensor(gpu_mindist) else gpu_mindist, np.float64)
         d_at = ((X64 - C64[gl]) ** 2).sum(1)
@@ -92,7 +104,8 @@ def check_labels(X64: np.ndarray, C64: np.ndarray, gpu_labels, dtype: str, gpu_m
 def centroid_slack(X64, labels_or, labels_gpu, C_or_next, counts_or) -> float:
     """Upper bound (relative to |C_or_next|_F) on the centroid change caused by
     moving the mismatched points from the oracle's clusters to the GPU's: each
-    move shifts two means by at most |x - mean| / (n - 1)."""
+    move shifts two means by at most |x - mean| / (n - 1).  Reported as a
+    diagnostic next to the centroid comparison; it never widens the gate."""
     gl = np.asarray(labels_gpu, np.int64)
     mism = np.nonzero(gl != labels_or)[0]
     if len(mism) == 0:

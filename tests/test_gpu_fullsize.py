@@ -31,7 +31,7 @@ def _bench_step(X, C):
     (rounded centroids, labels, new centroids, counts)."""
     C_dt, bias = fk.fk_prepare_centroids(C, X.dtype)
     labels = torch.empty(X.shape[:-1], dtype=torch.int32, device=X.device)
-    fk.fk_assign_prepared(X, C_dt, bias, labels)
+    fk.fk_assign_prepared(X, C_dt, bias, labels, xnorm=fk.fk_prepare_points(X))
     C_new = C.clone()
     counts = torch.empty(C.shape[:-1], dtype=torch.int32, device=X.device)
     fk.fk_update(X, labels, C_new, counts)

@@ -41,7 +41,80 @@ def test_assign_matches_oracle(shape, dtype):
     Xd, Cd = X.to(DEV), C.to(DEV)
     labels, mind = fk.fk_assign(Xd, Cd, want_mindist=True)
     fk.fk_sync()
-    check_labels(f64(X), f64(C), labels, dtype, gpu_mindist=mind)
+    check_labels(f64(X), f64(C), labels, dtype, gpu_mindist=mind, case=f"assign {N}x{D}x{K} {dtype}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("path", [1, 2])
+def test_near_ties_are_decided_exactly(dtype, path):
+    """Centroids in pairs one rounding step apart (and exact duplicates): many
+    points have two candidates whose distances differ by less than the fp32
+    error of the kernels' scores.  The listed near-ties are re-decided in
+    fp64 exactly as the oracle computes, so every label equals the oracle's."""
+    if dtype == "f32" and path == 1:
+        pytest.skip("fp32 runs on the CUDA-core kernel only")
+    g = torch.Generator().manual_seed(21)
+    N, D, half = 6000, 128, 300
+    base = (torch.randn(half, D, generator=g) * 2.0 + 3.0).to(TORCH_DT[dtype])
+    twin = base.clone()
+    # move one coordinate of each twin by one step of the input type
+    bits = twin.view(torch.int16 if dtype != "f32" else torch.int32)
+    col = torch.randint(0, D, (half,), generator=g)
+    bits[torch.arange(half), col] += 1
+    C = torch.cat([base, twin, base[:40]])  # and 40 exact duplicates
+    idx = torch.randint(0, C.shape[0], (N,), generator=g)
+    X = (C[idx].float() + 0.05 * torch.randn(N, D, generator=g)).to(TORCH_DT[dtype])
+    try:
+        fk.fk_set_assign_path(path)
+        labels, mind = fk.fk_assign(X.to(DEV), C.to(DEV), want_mindist=True)
+        fk.fk_sync()
+    finally:
+        fk.fk_set_assign_path(0)
+    st = check_labels(f64(X), f64(C), labels, dtype, gpu_mindist=mind, exact=True,
+                      case=f"near-tie pairs {dtype} path {path}")
+    assert st["near_tie_points"] > 0
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_full_comparison_when_three_chunks_tie(dtype):
+    """Every centroid of one group of five is an exact copy, placed in five
+    different 32-centroid chunks: points near that group tie five ways, so
+    the kernels list them for a comparison with every centroid; the label is
+    the lowest index of the group, as in the oracle."""
+    g = torch.Generator().manual_seed(33)
+    N, D, K = 4000, 128, 700
+    C = (torch.randn(K, D, generator=g) * 3.0).to(TORCH_DT[dtype])
+    group = [37, 100, 260, 450, 699]
+    C[group] = C[37].clone()
+    X = (C[torch.randint(0, K, (N,), generator=g)].float() + 0.05 * torch.randn(N, D, generator=g))
+    X[: N // 2] = (C[37].float() + 0.05 * torch.randn(N // 2, D, generator=g))
+    X = X.to(TORCH_DT[dtype])
+    labels, mind = fk.fk_assign(X.to(DEV), C.to(DEV), want_mindist=True)
+    fk.fk_sync()
+    check_labels(f64(X), f64(C), labels, dtype, gpu_mindist=mind, exact=True,
+                 case=f"five-way ties {dtype}")
+    assert not torch.isin(labels.cpu(), torch.tensor(group[1:], dtype=torch.int32)).any()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_prepared_points_and_assign(dtype):
+    """fk_prepare_points gives |x|^2 (fp32 sums of exact squares); the
+    prepared assignment with and without it gives the same labels."""
+    X, C0 = mixture(5000, 128, 600, dtype, seed=8, cfg="embed_f16")
+    Xd = X.to(DEV)
+    xn = fk.fk_prepare_points(Xd)
+    ref = (f64(X) ** 2).sum(1)
+    np.testing.assert_allclose(f64(xn), ref, rtol=2 * 128 * 2.0**-24, atol=0)
+    C_dt, bias = fk.fk_prepare_centroids(C0.to(DEV), TORCH_DT[dtype])
+    l1 = torch.empty(5000, dtype=torch.int32, device=DEV)
+    l2 = torch.empty_like(l1)
+    m1 = torch.empty(5000, device=DEV)
+    m2 = torch.empty_like(m1)
+    fk.fk_assign_prepared(Xd, C_dt, bias, l1, m1, xnorm=xn)
+    fk.fk_assign_prepared(Xd, C_dt, bias, l2, m2)
+    fk.fk_sync()
+    assert torch.equal(l1, l2)
+    check_labels(f64(X), f64(C_dt), l1, dtype, gpu_mindist=m1, exact=True, case=f"prepared points {dtype}")
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
@@ -201,9 +274,11 @@ def test_lloyd_step_by_step(cfg, N, K, iters, nc):
         C_next, lab, mind, _, counts = oracle.lloyd_step(X64, C, s.dtype)
         Cg = torch.from_numpy(C.astype(np.float32)).to(DEV)
         Cg, labels, gmind, gcounts = fk.fk_lloyd(Xd, Cg, 1, want_mindist=True)
-        check_labels(X64, oracle.round_to(s.dtype, C), labels, s.dtype, gpu_mindist=gmind)
-        slack = centroid_slack(X64, lab, labels.cpu().numpy(), C_next, counts)
-        check_centroids(Cg, C_next, tol=1e-4 + slack)
+        st = check_labels(X64, oracle.round_to(s.dtype, C), labels, s.dtype, gpu_mindist=gmind,
+                          case=f"lloyd {cfg} N={N} K={K} step {t}")
+        # the gate: the oracle's centroids from the oracle's labels, flat 1e-4
+        st["centroid_rel_l2"] = check_centroids(Cg, C_next)
+        st["slack"] = centroid_slack(X64, lab, labels.cpu().numpy(), C_next, counts)  # diagnostic only
         assert int(gcounts.sum()) == N
         assert torch.equal(gcounts.cpu().long(), torch.bincount(labels.cpu().long(), minlength=K))
         C = C_next
@@ -220,7 +295,8 @@ def test_lloyd_trajectory_matches_oracle(cfg, N, K, iters, nc):
     out = oracle.lloyd(f64(w.X), f64(w.C0), iters, s.dtype)
     check_centroids(C, out["C"])
     Cprev = oracle.lloyd(f64(w.X), f64(w.C0), iters - 1, s.dtype)["C"] if iters > 1 else f64(w.C0)
-    check_labels(f64(w.X), oracle.round_to(s.dtype, Cprev), labels, s.dtype, gpu_mindist=mind)
+    check_labels(f64(w.X), oracle.round_to(s.dtype, Cprev), labels, s.dtype, gpu_mindist=mind,
+                 case=f"lloyd trajectory {cfg} N={N} K={K}")
     assert int(counts.sum()) == N
 
 
@@ -340,4 +416,4 @@ def test_launch_counter_counts_kernels():
     n0 = fk.fk_launch_count()
     fk.fk_assign(X, X[:300].clone())
     fk.fk_sync()
-    assert fk.fk_launch_count() - n0 == 2  # norms + tensor-core assign
+    assert fk.fk_launch_count() - n0 == 3  # norms + tensor-core assign + near-tie re-decision

@@ -165,6 +165,31 @@ def pin_invariants(lib):
     assert all(b <= a * (1 + 1e-12) for a, b in zip(h, h[1:]))
 
 
+def pin_objective(lib):
+    # hand-worked: the 1-D case above, each point against its nearest centroid:
+    # J = 0 + 1 + 1 + 0 + 16 = 18
+    X = np.array([[0.0], [1.0], [9.0], [10.0], [4.0]])
+    C = np.array([[0.0], [10.0]])
+    assert oracle.objective(X, np.array([0, 0, 1, 1, 0], np.int32), C, lib) == 18.0
+    # labels need not be the nearest: every point on centroid 1 gives
+    # 100 + 81 + 1 + 0 + 36 = 218
+    assert oracle.objective(X, np.ones(5, np.int32), C, lib) == 218.0
+    # 2-D, worked by hand: (1,2)->(4,6): 25; (0,0)->(1,-1): 2; (3,3)->(4,6): 10
+    X2 = np.array([[1.0, 2.0], [0.0, 0.0], [3.0, 3.0]])
+    C2 = np.array([[4.0, 6.0], [1.0, -1.0]])
+    assert oracle.objective(X2, np.array([0, 1, 0], np.int32), C2, lib) == 37.0
+    # brute force with numpy on random data and random (not nearest) labels
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((700, 9))
+    C = rng.standard_normal((23, 9))
+    lab = rng.integers(0, 23, 700).astype(np.int32)
+    ref = float(((X - C[lab]) ** 2).sum())
+    assert oracle.objective(X, lab, C, lib) == pytest.approx(ref, rel=1e-12)
+    # with the nearest labels it equals the sum of the assignment's distances
+    lab, mind, _ = oracle.assign(X, C, lib)
+    assert oracle.objective(X, lab, C, lib) == pytest.approx(float(mind.sum()), rel=1e-12)
+
+
 def pin_planted(lib):
     rng = np.random.default_rng(8)
     K, D, per = 12, 6, 40
@@ -180,7 +205,7 @@ def pin_planted(lib):
 
 
 PINS = [pin_vq, pin_sklearn_step, pin_hand_1d, pin_ties, pin_k1_mean, pin_prefix_identity,
-        pin_permutation, pin_empty_cluster, pin_invariants, pin_planted]
+        pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_planted]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -217,22 +242,49 @@ def test_round_to_f16_matches_torch():
     assert np.array_equal(oracle.round_to("f16", v), ref)
 
 
-def test_lloyd_loop_matches_manual_steps(oracle_lib):
+def test_lloyd_loop_against_independent_steps(oracle_lib):
+    """oracle.lloyd against other implementations of each step: torch's
+    round-to-nearest-even casts (fp32 master, then bf16), scipy's vq for the
+    nearest centroid and numpy for the means (empty clusters keep the master)."""
+    import torch
+    from scipy.cluster.vq import vq
     rng = np.random.default_rng(11)
-    X = oracle.round_to("bf16", rng.standard_normal((300, 8)))
-    out = oracle.lloyd(X, X[:5], 3, "bf16", oracle_lib)
-    C = X[:5].copy()
+    X = torch.from_numpy(rng.standard_normal((300, 8))).to(torch.bfloat16).double().numpy()
+    K = 5
+    out = oracle.lloyd(X, X[:K], 3, "bf16", oracle_lib)
+    C32 = torch.from_numpy(X[:K]).float()
     for _ in range(3):
-        Cr = oracle.round_to("bf16", C)
-        lab, mind, _ = oracle.assign(X, Cr, oracle_lib)
-        Cn, _ = oracle.update(X, lab, 5, C, oracle_lib)
-        C = Cn.astype(np.float32).astype(np.float64)
-    assert np.array_equal(out["C"], C) and np.array_equal(out["labels"], lab)
+        Cr = C32.to(torch.bfloat16).double().numpy()
+        lab, dist = vq(X, Cr)
+        nxt = C32.clone()
+        for k in range(K):
+            if (lab == k).any():
+                nxt[k] = torch.from_numpy(X[lab == k].mean(0)).float()
+        C32 = nxt
+    assert np.array_equal(out["labels"], lab.astype(np.int32))
+    np.testing.assert_allclose(out["C"], C32.double().numpy(), rtol=0, atol=2e-7)
+    np.testing.assert_allclose(out["mindist"], dist ** 2, rtol=1e-12, atol=1e-12)
+
+
+def test_lloyd_f64_matches_sklearn(oracle_lib):
+    """Several fp64 Lloyd iterations against scikit-learn's Lloyd from the
+    same initial centroids (a case without empty clusters)."""
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(13)
+    X = rng.standard_normal((800, 6)) + 4.0 * rng.integers(0, 3, (800, 1))
+    C0 = X[:8].copy()
+    out = oracle.lloyd(X, C0, 4, "f64", oracle_lib)
+    assert out["counts"].min() > 0
+    km = KMeans(n_clusters=8, init=C0, n_init=1, max_iter=4, algorithm="lloyd", tol=0.0).fit(X)
+    np.testing.assert_allclose(out["C"], km.cluster_centers_, rtol=1e-10, atol=1e-12)
 
 
 # ---------------------------------------------------------------- golden ---
 def test_golden_fixture(oracle_lib):
-    """Regression pin: values written by tests/golden/make_golden.py (oracle only)."""
+    """Regression check, not a pin: the oracle against values an earlier build
+    of itself wrote (tests/golden/make_golden.py, oracle only).  It catches an
+    unintended change of the oracle's arithmetic; the pins above are what tie
+    the oracle to the definition."""
     import json
     import workloads
     path = os.path.join(HERE, "golden", "tiny_f32_n512_k16.json")
@@ -258,6 +310,11 @@ MUTANTS = [
     ("mean off by one", "out[j] = s[j] / (double)counts[k];", "out[j] = s[j] / (double)(counts[k] + 1);"),
     ("empty cluster zeroed", "for (int j = 0; j < D; ++j) out[j] = prev[j];",
      "for (int j = 0; j < D; ++j) out[j] = 0.0;"),
+    ("objective on the wrong centroid", "C + (size_t)labels[i] * (size_t)D, D);",
+     "C + (size_t)(labels[i] + 1 < 0 ? 0 : 0) * (size_t)D, D);"),
+    ("objective drops the last point", "for (int64_t i = 0; i < N; ++i)\n        J +=",
+     "for (int64_t i = 0; i + 1 < N; ++i)\n        J +="),
+    ("objective not accumulated", "J += sqdist(", "J = sqdist("),
     ("last point dropped", "for (int64_t i = 0; i < N; ++i) {\n        int32_t k = labels[i];",
      "for (int64_t i = 0; i + 1 < N; ++i) {\n        int32_t k = labels[i];"),
 ]
