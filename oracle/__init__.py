@@ -51,6 +51,8 @@ def _bind(lib):
     lib.oracle_assign.restype = None
     lib.oracle_update.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, dp, lp]
     lib.oracle_update.restype = ctypes.c_int
+    lib.oracle_label_dist.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp, dp]
+    lib.oracle_label_dist.restype = None
     lib.oracle_objective.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp]
     lib.oracle_objective.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
@@ -95,6 +97,75 @@ def assign(X, C, lib=None):
         lib.oracle_assign(_p(X, ctypes.c_double), N, D, _p(C, ctypes.c_double), K,
                           _p(labels, ctypes.c_int32), _p(mind, ctypes.c_double),
                           _p(second, ctypes.c_double))
+    return labels, mind, second
+
+
+def label_dist(X, labels, C, lib=None):
+    """|x_i - c_{labels[i]}|^2 per row, the sum oracle_assign forms (fp64)."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    labels = np.ascontiguousarray(labels, dtype=np.int32)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    out = np.zeros(X.shape[0], np.float64)
+    if X.shape[0]:
+        lib.oracle_label_dist(_p(X, ctypes.c_double), _p(labels, ctypes.c_int32), X.shape[0], X.shape[1],
+                              _p(C, ctypes.c_double), _p(out, ctypes.c_double))
+    return out
+
+
+def assign_screened(X, C, lib=None, block_elems=1 << 25, margin: float = 4.0):
+    """``assign`` reached faster on large inputs, with the same labels and
+    mindist.
+
+    A library matrix product (torch on the CPU, fp32) gives every expanded
+    distance e_k = |c_k|^2 - 2<x, c_k> (the |x|^2 term is common to a row) to
+    within delta = margin (D + 8) 2^-24 (|x|^2 + max_k |c_k|^2), margin = 4: a
+    generous form of
+    the classical bound on the rounding of a length-D dot product and of the
+    sums of squares.  A centroid whose e_k exceeds the row minimum by more
+    than 2 delta is farther than the nearest one, so it cannot be the
+    answer.  A row with one centroid left gets it, and its distance from
+    ``label_dist`` (the oracle's own sum); every row with more left goes
+    whole through ``assign``.  ``second`` is ``assign``'s for those rows and
+    the second-smallest screened distance (|x|^2 added back) otherwise."""
+    import torch
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    N, D = X.shape
+    K = C.shape[0]
+    labels = np.zeros(N, np.int32)
+    mind = np.zeros(N, np.float64)
+    second = np.full(N, np.inf)
+    if N == 0:
+        return labels, mind, second
+    C32 = torch.from_numpy(C.astype(np.float32))
+    cn = (C * C).sum(1)
+    cn32 = torch.from_numpy(cn.astype(np.float32))
+    cmax = float(cn.max())
+    xn_all = np.einsum("ij,ij->i", X, X)
+    rows = max(1, min(N, block_elems // max(K, 1)))
+    multi = []
+    Ebuf = torch.empty((rows, K), dtype=torch.float32)  # reused: fresh pages for every block cost more than the product
+    for r0 in range(0, N, rows):
+        r1 = min(N, r0 + rows)
+        Xb = torch.from_numpy(X[r0:r1].astype(np.float32))
+        E = torch.addmm(cn32.unsqueeze(0), Xb, C32.t(), beta=1.0, alpha=-2.0, out=Ebuf[: r1 - r0])
+        delta = margin * (D + 8) * 2.0 ** -24 * (xn_all[r0:r1] + cmax)
+        if K > 1:
+            v, i = torch.topk(E, 2, dim=1, largest=False)
+            v = v.double().numpy()
+            labels[r0:r1] = i[:, 0].numpy()
+            second[r0:r1] = v[:, 1] + xn_all[r0:r1]
+            # more than one centroid within 2 delta of the row minimum
+            multi.append(np.nonzero(v[:, 1] <= v[:, 0] + 2.0 * delta)[0] + r0)
+    multi = np.concatenate(multi) if multi else np.zeros(0, np.int64)
+    mind[:] = label_dist(X, labels, C, lib)  # rows with several candidates are redone below
+    if len(multi):
+        lm, dm, sm = assign(X[multi], C, lib)
+        labels[multi] = lm
+        mind[multi] = dm
+        second[multi] = sm
     return labels, mind, second
 
 
@@ -162,14 +233,15 @@ def round_to(dtype: str, a) -> np.ndarray:
 
 
 # ------------------------------------------------------------------ Lloyd --
-def lloyd_step(X, C_master, dtype: str, lib=None):
+def lloyd_step(X, C_master, dtype: str, lib=None, screened: bool = False):
     """One Lloyd iteration from fp32 (or fp64 when dtype == "f64") master centroids.
 
     Assignment uses the master rounded to ``dtype``; the update's empty-cluster
-    rule keeps the master value.  Returns (C_next master, labels, mindist,
-    second, counts)."""
+    rule keeps the master value.  ``screened`` takes the assignment from
+    ``assign_screened`` (same labels, faster on large inputs).  Returns
+    (C_next master, labels, mindist, second, counts)."""
     Cr = round_to(dtype, C_master)
-    labels, mind, second = assign(X, Cr, lib)
+    labels, mind, second = (assign_screened if screened else assign)(X, Cr, lib)
     Cn, counts = update(X, labels, Cr.shape[0], np.asarray(C_master, np.float64), lib)
     Cn = Cn if dtype == "f64" else to_f32(Cn).astype(np.float64)
     return Cn, labels, mind, second, counts

@@ -107,6 +107,15 @@ int oracle_update(const double *X, const int32_t *labels, int64_t N, int D, int 
     return 0;
 }
 
+/* Squared distance of each point to its given centroid:
+ * out[i] = |x_i - c_{labels[i]}|^2, the same sum as oracle_assign forms. */
+void oracle_label_dist(const double *X, const int32_t *labels, int64_t N, int D, const double *C,
+                       double *out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i)
+        out[i] = sqdist(X + (size_t)i * (size_t)D, C + (size_t)labels[i] * (size_t)D, D);
+}
+
 /* Lloyd objective J = sum_i |x_i - c_{labels[i]}|^2. */
 double oracle_objective(const double *X, const int32_t *labels, int64_t N, int D,
                         const double *C) {

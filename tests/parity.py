@@ -60,17 +60,26 @@ def fp32_separation(D: int) -> float:
 
 
 def check_labels(X64: np.ndarray, C64: np.ndarray, gpu_labels, dtype: str, gpu_mindist=None,
-                 exact: bool = False, max_frac: float = MAX_MISMATCH_FRAC, case: str = ""):
+                 exact: bool = False, max_frac: float = MAX_MISMATCH_FRAC, case: str = "",
+                 screened: bool = False, oracle_out=None):
     """Compare GPU labels (and mindist) with the oracle on the same rounded inputs.
 
+    ``screened`` takes the oracle's labels from ``oracle.assign_screened``
+    (identical to ``oracle.assign``, faster on large inputs); ``oracle_out``
+    passes an (labels, mindist, second) triple the oracle already computed.
     Returns a dict of statistics (also recorded in ``STATS`` when ``case`` is
     given); raises AssertionError when the bar is missed."""
     gl = np.asarray(gpu_labels.cpu() if torch.is_tensor(gpu_labels) else gpu_labels).astype(np.int64)
-    lab, mind, second = oracle.assign(X64, C64)
+    if oracle_out is not None:
+        lab, mind, second = oracle_out
+    else:
+        lab, mind, second = (oracle.assign_screened if screened else oracle.assign)(X64, C64)
     N = len(lab)
     assert gl.min(initial=0) >= 0 and gl.max(initial=0) < C64.shape[0], "label out of range"
     mism = np.nonzero(gl != lab)[0]
-    scale = (X64 ** 2).sum(1) + (C64[lab] ** 2).sum(1)
+    cn = np.einsum("ij,ij->i", C64, C64)
+    xn = np.einsum("ij,ij->i", X64, X64)
+    scale = xn + cn[lab]
     gap = second - mind
     stats = {"N": N, "mismatch": int(len(mism)),
              "near_tie_points": int((gap <= BAND[dtype] * scale).sum()), "fp32_ties": 0}
@@ -93,9 +102,9 @@ def check_labels(X64: np.ndarray, C64: np.ndarray, gpu_labels, dtype: str, gpu_m
                                            f"{max_frac:.2%} of {N} rows")
     if gpu_mindist is not None:
         gm = np.asarray(gpu_mindist.cpu() if torch.is_tensor(gpu_mindist) else gpu_mindist, np.float64)
-        d_at = ((X64 - C64[gl]) ** 2).sum(1)
+        d_at = oracle.label_dist(X64, gl.astype(np.int32), C64)
         err = np.abs(gm - d_at)
-        tol = MINDIST_TOL[dtype] * ((X64 ** 2).sum(1) + (C64[gl] ** 2).sum(1)) + 1e-30
+        tol = MINDIST_TOL[dtype] * (xn + cn[gl]) + 1e-30
         assert np.all(err <= tol), f"mindist off by {float((err / tol).max()):.3g} x tolerance"
         assert np.all(gm >= 0)
     return stats

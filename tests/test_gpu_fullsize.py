@@ -1,14 +1,21 @@
-"""Parity at the full sizes of the configured workloads.
+"""Parity at the full sizes of the configured workloads, one Lloyd step at a
+time, in bench.py's launch configuration (fk_prepare_centroids,
+fk_prepare_points once, fk_assign_prepared and fk_update on inputs resident in
+HBM; the out-of-core case runs fk_lloyd_ooc from pinned host memory).
 
-Each case runs one Lloyd step the way bench.py times it: fk_prepare_centroids,
-fk_assign_prepared and fk_update on inputs resident in HBM; the out-of-core
-case runs fk_lloyd_ooc from pinned host memory.  The oracle cannot afford all
-N x K distances at these sizes, so it checks:
-  * the labels of a seeded sample of rows, against oracle.assign on the same
-    rounded rows and centroids (the usual near-tie rule);
-  * the counts, against a bincount of the GPU's labels (bit-exact);
-  * the centroids of a sample of clusters (the largest one included), against
-    oracle.update on their members, and an empty cluster keeping its centroid.
+* Embedding (2^20 x 128, K = 1024, 20 iterations) and batched (32 problems of
+  32,768 x 128, K = 256, 10 iterations): the oracle runs its own trajectory
+  over every row (its screened assignment, which gives the plain oracle's
+  labels exactly), and every GPU step starts from the oracle's centroids of
+  that step.  Labels of all rows, counts and the next centroids are compared.
+* Zipf (2^23 x 128, K = 65,536): one oracle step over every row needs about
+  1.4e14 fp64 flops, so at this size the GPU's own trajectory is checked
+  step by step for what holds at any size -- the labels of a seeded sample of
+  rows are the nearest of the centroids that step used (oracle, exact), the
+  counts are the label histogram, sampled clusters (the largest among them)
+  are the oracle's means of their members, and every empty cluster keeps its
+  centroid.  The oracle's own trajectory is compared over every row on the
+  same recipe at 2^19 rows and K = 4,096.
 """
 import numpy as np
 import pytest
@@ -17,80 +24,119 @@ import torch
 import distance_argmin_flashassign_b200 as fk
 import oracle
 import workloads
-from tests.parity import CENTROID_REL_L2, check_labels, f64, rel_l2
+from tests.parity import CENTROID_REL_L2, check_centroids, check_labels, f64, record, rel_l2
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 DEV = "cuda:0"
-DT = {"f16": torch.float16, "bf16": torch.bfloat16}
-SAMPLE_ROWS = 2048
+SAMPLE_ROWS = 4096
 SAMPLE_CLUSTERS = 16
 
 
-def _bench_step(X, C):
-    """One Lloyd step in bench.py's launch configuration; returns
-    (rounded centroids, labels, new centroids, counts)."""
-    C_dt, bias = fk.fk_prepare_centroids(C, X.dtype)
-    labels = torch.empty(X.shape[:-1], dtype=torch.int32, device=X.device)
-    fk.fk_assign_prepared(X, C_dt, bias, labels, xnorm=fk.fk_prepare_points(X))
-    C_new = C.clone()
-    counts = torch.empty(C.shape[:-1], dtype=torch.int32, device=X.device)
-    fk.fk_update(X, labels, C_new, counts)
-    torch.cuda.synchronize()
-    return C_dt, labels, C_new, counts
+class BenchStep:
+    """One Lloyd step as bench.py times it, on inputs resident in HBM."""
+
+    def __init__(self, X):
+        self.X = X
+        self.xnorm = fk.fk_prepare_points(X)
+
+    def __call__(self, C):
+        """C: fp32 master centroids on the device.  Returns (rounded
+        centroids, labels, new centroids, counts)."""
+        X = self.X
+        C_dt, bias = fk.fk_prepare_centroids(C, X.dtype)
+        labels = torch.empty(X.shape[:-1], dtype=torch.int32, device=X.device)
+        fk.fk_assign_prepared(X, C_dt, bias, labels, xnorm=self.xnorm)
+        C_new = C.clone()
+        counts = torch.empty(C.shape[:-1], dtype=torch.int32, device=X.device)
+        fk.fk_update(X, labels, C_new, counts)
+        fk.fk_sync()
+        return C_dt, labels, C_new, counts
 
 
-def _check_problem(X, C_prev, C_dt, labels, C_new, counts, dtype, rng):
-    """Sampled checks of one problem (X N x D on the device, the rest 1-problem views)."""
-    N, D = X.shape
-    K = C_prev.shape[0]
-    # labels of sampled rows against the oracle on the same rounded values
-    rows = np.sort(rng.choice(N, size=min(SAMPLE_ROWS, N), replace=False))
-    ridx = torch.as_tensor(rows, device=X.device)
-    X64 = f64(X[ridx])
-    stats = check_labels(X64, f64(C_dt), labels[ridx], dtype)
-    # counts: exact, from the labels
-    lab = labels.long()
-    assert int(counts.sum()) == N
-    assert torch.equal(counts, torch.bincount(lab, minlength=K).to(torch.int32))
-    # centroids of sampled clusters: the largest, random non-empty ones, and an empty one
-    cnt = counts.cpu().numpy()
-    nonempty = np.nonzero(cnt)[0]
-    ks = {int(np.argmax(cnt))}
-    ks.update(int(k) for k in rng.choice(nonempty, size=min(SAMPLE_CLUSTERS, len(nonempty)), replace=False))
-    ks = np.array(sorted(ks))
-    kidx = torch.as_tensor(ks, device=X.device)
-    member = torch.isin(lab, kidx)
-    Xm = f64(X[member])
-    remap = torch.full((K,), -1, dtype=torch.long, device=X.device)
-    remap[kidx] = torch.arange(len(ks), device=X.device)
-    lm = remap[lab[member]].cpu().numpy().astype(np.int32)
-    C_or, cnt_or = oracle.update(Xm, lm, len(ks), f64(C_prev[kidx]))
-    assert np.array_equal(cnt_or, cnt[ks])
-    r = rel_l2(f64(C_new[kidx]), C_or)
-    assert r <= CENTROID_REL_L2, f"sampled-centroid rel-L2 {r:.3g}"
-    empty = np.nonzero(cnt == 0)[0]
-    if len(empty):
-        k = int(empty[0])
-        assert torch.equal(C_new[k], C_prev[k]), "an empty cluster must keep its centroid"
-    return stats, r
+def _oracle_trajectory_check(name, X, C0, dtype, iters, problem_ids=None):
+    """Every step: GPU from the oracle's C_t against the oracle's step."""
+    step = BenchStep(X)
+    batched = X.dim() == 3
+    probs = list(range(X.shape[0])) if batched else [None]
+    X64 = [f64(X[b]) if batched else f64(X) for b in probs]
+    C = [f64(C0[b]) if batched else f64(C0) for b in probs]
+    for t in range(iters):
+        Cg = torch.from_numpy(np.stack(C) if batched else C[0]).float().to(DEV)
+        _, labels, C_new, counts = step(Cg)
+        for i, b in enumerate(probs):
+            C_next, lab, mind, second, cnt = oracle.lloyd_step(X64[i], C[i], dtype, screened=True)
+            gl = labels[b] if batched else labels
+            st = check_labels(X64[i], oracle.round_to(dtype, C[i]), gl, dtype, oracle_out=(lab, mind, second),
+                              case=f"full size {name} step {t}" + (f" problem {b}" if batched else ""))
+            gc = (counts[b] if batched else counts).cpu().numpy()
+            assert np.array_equal(gc, cnt), "counts differ from the oracle's"
+            st["centroid_rel_l2"] = check_centroids(C_new[b] if batched else C_new, C_next)
+            C[i] = C_next
 
 
-@pytest.mark.parametrize("name", ["embed_f16", "zipf_bf16"])
-def test_full_size_single_problem(name):
-    s = workloads.spec(name)
+def test_full_size_embedding_trajectory():
+    s = workloads.spec("embed_f16")
     w = workloads.make(s, device=DEV)
-    C_dt, labels, C_new, counts = _bench_step(w.X, w.C0.clone())
-    stats, r = _check_problem(w.X, w.C0, C_dt, labels, C_new, counts, s.dtype, np.random.default_rng(11))
-    assert stats["N"] == SAMPLE_ROWS
+    _oracle_trajectory_check("embed_f16", w.X, w.C0, s.dtype, s.iters)
 
 
-def test_full_size_batched():
+def test_full_size_batched_trajectory():
     s = workloads.spec("batched_bf16")
     w = workloads.make(s, device=DEV)
-    C_dt, labels, C_new, counts = _bench_step(w.X, w.C0.clone())
-    rng = np.random.default_rng(12)
-    for b in (0, s.B // 2, s.B - 1):  # first, middle and last problem of the one launch
-        _check_problem(w.X[b], w.C0[b], C_dt[b], labels[b], C_new[b], counts[b], s.dtype, rng)
+    _oracle_trajectory_check("batched_bf16", w.X, w.C0, s.dtype, s.iters)
+
+
+def test_zipf_reduced_trajectory():
+    """The Zipf recipe at 2^19 rows and K = 4,096 (as many centres), every
+    row compared against the oracle's own trajectory for the configured 10
+    iterations."""
+    s = workloads.spec("zipf_bf16", N=1 << 19, K=4096, n_centers=4096)
+    w = workloads.make(s, device=DEV)
+    _oracle_trajectory_check("zipf_bf16 2^19 x 4096", w.X, w.C0, s.dtype, s.iters)
+
+
+def test_zipf_full_size_steps():
+    s = workloads.spec("zipf_bf16")
+    w = workloads.make(s, device=DEV)
+    X = w.X
+    N, K = s.N, s.K
+    step = BenchStep(X)
+    rng = np.random.default_rng(11)
+    C = w.C0.clone()
+    for t in range(s.iters):
+        _, labels, C_new, counts = step(C)
+        # labels of sampled rows: the nearest of the centroids this step used
+        rows = np.sort(rng.choice(N, size=SAMPLE_ROWS, replace=False))
+        ridx = torch.as_tensor(rows, device=DEV)
+        st = check_labels(f64(X[ridx]), oracle.round_to(s.dtype, f64(C)), labels[ridx], s.dtype, screened=True,
+                          case=f"full size zipf_bf16 step {t} (sampled rows)")
+        # counts: the label histogram, exactly
+        lab = labels.long()
+        assert int(counts.sum()) == N
+        assert torch.equal(counts, torch.bincount(lab, minlength=K).to(torch.int32))
+        # sampled clusters are the means of their members; the largest one at
+        # the first and the last step
+        cnt = counts.cpu().numpy()
+        nonempty = np.nonzero(cnt)[0]
+        ks = {int(k) for k in rng.choice(nonempty, size=min(SAMPLE_CLUSTERS, len(nonempty)), replace=False)}
+        if t in (0, s.iters - 1):
+            ks.add(int(np.argmax(cnt)))
+        ks = np.array(sorted(ks))
+        kidx = torch.as_tensor(ks, device=DEV)
+        member = torch.isin(lab, kidx)
+        remap = torch.full((K,), -1, dtype=torch.long, device=DEV)
+        remap[kidx] = torch.arange(len(ks), device=DEV)
+        C_or, cnt_or = oracle.update(f64(X[member]), remap[lab[member]].cpu().numpy().astype(np.int32), len(ks),
+                                     f64(C[kidx]))
+        assert np.array_equal(cnt_or, cnt[ks])
+        r = rel_l2(f64(C_new[kidx]), C_or)
+        assert r <= CENTROID_REL_L2, f"sampled-centroid rel-L2 {r:.3g}"
+        st["centroid_rel_l2"] = r
+        # every empty cluster keeps its centroid
+        empty = counts == 0
+        assert torch.equal(C_new[empty], C[empty])
+        st["empty_clusters"] = int(empty.sum())
+        C = C_new
 
 
 def test_out_of_core_large_chunks():
@@ -110,7 +156,8 @@ def test_out_of_core_large_chunks():
     rng = np.random.default_rng(13)
     rows = np.sort(rng.choice(N, size=SAMPLE_ROWS, replace=False))
     C64 = oracle.round_to("f16", C0.numpy())
-    check_labels(Xh[rows].double().numpy(), C64, lab_h[rows], "f16")
+    check_labels(Xh[rows].double().numpy(), C64, lab_h[rows], "f16", screened=True,
+                 case="out of core 2^24 rows (sampled rows)")
     assert int(cnt_h.sum()) == N
     assert torch.equal(cnt_h, torch.bincount(lab_h.long(), minlength=s.K).to(torch.int32))
     ks = np.sort(rng.choice(np.nonzero(cnt_h.numpy())[0], size=SAMPLE_CLUSTERS, replace=False))
@@ -121,3 +168,4 @@ def test_out_of_core_large_chunks():
                                  C0[ks].double().numpy())
     assert np.array_equal(cnt_or, cnt_h.numpy()[ks])
     assert rel_l2(Ch[ks].double().numpy(), C_or) <= CENTROID_REL_L2
+    record("out of core 2^24 rows (sampled clusters)", centroid_rel_l2=rel_l2(Ch[ks].double().numpy(), C_or))

@@ -218,6 +218,51 @@ def test_update_rejects_bad_label(oracle_lib):
         oracle.update(np.zeros((3, 2)), np.array([0, 2, 1], np.int32), 2, np.zeros((2, 2)), oracle_lib)
 
 
+# --------------------------------------------------------- screened assign --
+def _screen_cases():
+    rng = np.random.default_rng(14)
+    yield "normal", rng.standard_normal((3000, 64)), rng.standard_normal((300, 64))
+    X = rng.integers(-3, 4, (2000, 16)).astype(np.float64)
+    C = rng.integers(-3, 4, (120, 16)).astype(np.float64)
+    C[60:] = C[:60]  # every centroid twice: exact ties everywhere
+    yield "integer ties", X, C
+    import torch
+    base = (rng.standard_normal((200, 128)) * 2 + 3).astype(np.float32)
+    twin = torch.from_numpy(base).to(torch.bfloat16)
+    bits = twin.view(torch.int16)
+    bits[np.arange(200), rng.integers(0, 128, 200)] += 1
+    Cb = np.concatenate([torch.from_numpy(base).to(torch.bfloat16).double().numpy(), twin.double().numpy()])
+    Xb = torch.from_numpy(Cb[rng.integers(0, 400, 3000)] + 0.05 * rng.standard_normal((3000, 128))).to(
+        torch.bfloat16).double().numpy()
+    yield "one-ulp twins", Xb, Cb
+    yield "large offset", 1000.0 + 0.01 * rng.standard_normal((2000, 32)), 1000.0 + 0.01 * rng.standard_normal((50, 32))
+    yield "K = 1", rng.standard_normal((100, 8)), rng.standard_normal((1, 8))
+
+
+@pytest.mark.parametrize("case", list(_screen_cases()), ids=lambda c: c[0])
+def test_screened_assign_equals_plain(case, oracle_lib):
+    """assign_screened must return exactly assign's labels and distances
+    (brute force on the same inputs), including exact ties, near-ties one
+    bf16 step apart and inputs whose expanded distances cancel badly."""
+    _, X, C = case
+    lab, mind, second = oracle.assign(X, C, oracle_lib)
+    l2, m2, s2 = oracle.assign_screened(X, C, oracle_lib, block_elems=1 << 14)
+    assert np.array_equal(lab, l2)
+    assert np.array_equal(mind, m2)
+    if C.shape[0] > 1:
+        np.testing.assert_allclose(s2, second, rtol=1e-4, atol=1e-6 * float(np.abs(second).max()))
+
+
+def test_screened_assign_margin_matters(oracle_lib):
+    """With no rounding margin the screening decides near-ties in fp32 and
+    disagrees with the plain oracle: the equality pin above would catch a
+    screening that dropped its margin."""
+    _, X, C = [c for c in _screen_cases() if c[0] == "one-ulp twins"][0]
+    lab, _, _ = oracle.assign(X, C, oracle_lib)
+    l0, _, _ = oracle.assign_screened(X, C, oracle_lib, margin=0.0)
+    assert not np.array_equal(lab, l0)
+
+
 # ------------------------------------------------------------- rounding ----
 def test_bf16_rounding_nearest_even():
     import torch
