@@ -5,15 +5,23 @@ One step = one pass of the whole hot path on the embedding workload
 headline metric is quoted on):
 
     fk_prepare_centroids  (round fp32 centroids to fp16, bias -|c|^2/2)
-    fk_assign_prepared    (tcgen05 FlashAssign: distances + online argmin)
+    fk_assign_prepared    (tcgen05 FlashAssign: distances + online argmin,
+                           then the exact re-decision of near-ties)
     fk_update             (sort-inverse update: radix sort, segment offsets,
                            segmented sums, divide)
 
 all through the C ABI, inputs resident in HBM (X = 256 MiB, larger than the
-126 MB L2, so no flush is needed between steps).
+126 MB L2, so no flush is needed between steps); |x|^2 of the points is
+prepared once (fk_prepare_points), as X does not change between iterations.
+
+On one GPU the line also carries "workloads": the same measurement of the
+other configured workloads (tiny fp32, batched bf16, Zipf bf16) and the
+out-of-core one at 2^27 rows (--ooc-rows-all), each with its own rooflines
+against the measured and the spec peaks, its CPU baseline and its clocks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu] [--ooc-rows R]
+                    [--workload NAME] [--no-e2e] [--no-cpu] [--no-all]
+                    [--ooc-rows R] [--ooc-rows-all R]
 
 --workload ooc_f16 runs the out-of-core workload instead (one GPU): X in
 pinned host memory, streamed through fk_lloyd_ooc in the configured 64 Mi-row
@@ -212,26 +220,26 @@ def build_inputs(name: str, device, seed: int):
     return s, w
 
 
-def bench_gpu(args):
+# Spec peaks of a B200 (the stricter denominators, reported next to the
+# measured ones): dense fp16/bf16 tensor throughput and HBM3e bandwidth.
+SPEC_P16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
+
+def measure(args, name: str, fk, dev, world: int, rank: int, steps: int, warmup: int, cpu_budget: float,
+            seed: int):
+    """Time `steps` Lloyd iterations of workload `name` resident in HBM: one
+    step = fk_prepare_centroids + fk_assign_prepared (the assignment kernel
+    and the exact re-decision of near-ties) + fk_update, all through the C
+    ABI, with |x|^2 prepared once (X does not change between iterations).
+    Returns the workload's JSON fields and the raw timings."""
     import torch
-
-    import distance_argmin_flashassign_b200 as fk
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    s, w = build_inputs(args.workload, dev, seed=rank)
+    s, w = build_inputs(name, dev, seed)
     dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[s.dtype]
     X = w.X
     B, N, D, K = s.B, s.N, s.D, s.K
     C = w.C0.clone()
     C_dt, bias = fk.fk_prepare_centroids(C, dt)
-    # |x|^2 of every point, once: X does not change between iterations
     xnorm = fk.fk_prepare_points(X) if dt != torch.float32 else None
     labels = torch.empty(((B, N) if B > 1 else (N,)), dtype=torch.int32, device=dev)
     counts = torch.empty(((B, K) if B > 1 else (K,)), dtype=torch.int32, device=dev)
@@ -248,15 +256,15 @@ def bench_gpu(args):
         if ev:
             ev[2].record(stream)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     fk.fk_sync()
     torch.cuda.synchronize(dev)
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     time.sleep(0.3)  # let the sampler start before the timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -264,7 +272,7 @@ def bench_gpu(args):
     n0 = fk.fk_launch_count()
     w0 = time.time()
     t_start.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -278,56 +286,102 @@ def bench_gpu(args):
     t_assign = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_update = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
 
-    value, t_max = aggregate(args.steps, elapsed, world, dev)
+    value, t_max = aggregate(steps, elapsed, world, dev)
     peaks, peak_kind = load_peaks()
     flops = 2.0 * B * N * K * D
     es = s.bytes_per_elem
+    assign_bytes = B * (N * D * es + K * D * es + 32 * K + 8 * N)
     upd_bytes = B * (N * D * es + 4 * N + K * (4 * D + 4))
     tflops = flops / (t_assign * 1e-3) / 1e12
     gbs = upd_bytes / (t_update * 1e-3) / 1e9
+    stage = "assignment stage: assign kernel + exact near-tie re-decision kernel"
     if s.dtype == "f32":
         # fp32 runs on the CUDA-core kernel: bound by the FP32 FMA pipes, whose
         # peak is derived from the unit counts and the maximum SM clock
         props = torch.cuda.get_device_properties(dev)
         fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_GHZ / 1e3
-        roofline = {"bound": "alu", "kernel": "assign_simt_kernel", "achieved": round(tflops, 3),
+        roofline = {"bound": "alu", "kernel": "assign_simt_kernel", "stage": stage, "achieved": round(tflops, 3),
                     "peak": round(fp32_peak, 1), "unit": "TFLOP/s", "frac": round(tflops / fp32_peak, 4),
                     "peak_kind": f"fp32 FMA: {props.multi_processor_count} SMs x {FP32_LANES_PER_SM} lanes x "
                                  f"2 flop x {SM_MAX_GHZ} GHz (derived from unit counts and clock)",
                     "traffic": None, "ms_per_launch": round(t_assign, 5), "algorithmic_flops_per_launch": flops}
     else:
-        roofline = {"bound": "tensor", "kernel": "assign_tc_kernel", "achieved": round(tflops, 2),
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": round(tflops / peaks["bf16_tflops"], 4),
-                    "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
-                    "traffic": profiled_traffic(args.workload), "ms_per_launch": round(t_assign, 5),
-                    "algorithmic_flops_per_launch": flops}
+        ai = flops / assign_bytes
+        peak_meas = min(peaks["bf16_tflops"], ai * peaks["hbm_gbs"] / 1e3)
+        peak_spec = min(SPEC_P16_TFLOPS, ai * SPEC_HBM_GBS / 1e3)
+        bound = "tensor" if peak_meas >= peaks["bf16_tflops"] else "hbm"
+        roofline = {"bound": bound, "kernel": "assign_tc_kernel", "stage": stage, "achieved": round(tflops, 2),
+                    "peak": round(peak_meas, 1), "unit": "TFLOP/s", "frac": round(tflops / peak_meas, 4),
+                    "peak_kind": (f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)" if bound == "tensor" else
+                                  f"arithmetic intensity {ai:.0f} flop/B x {peak_kind} copy bandwidth "
+                                  "(below the tensor peak)"),
+                    "peak_spec": round(peak_spec, 1), "frac_spec": round(tflops / peak_spec, 4),
+                    "traffic": profiled_traffic(name), "ms_per_launch": round(t_assign, 5),
+                    "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": assign_bytes}
     roofline_update = {"bound": "hbm", "kernels": "fk_update (sort, offsets, segsum, finalize)",
                        "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peak_kind} copy",
+                       "peak_spec": SPEC_HBM_GBS, "frac_spec": round(gbs / SPEC_HBM_GBS, 4),
                        "ms_per_call": round(t_update, 5), "algorithmic_bytes_per_call": upd_bytes}
-
-    out = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 5), "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
-           "config": {"workload": args.workload, "N": N, "D": D, "K": K, "B": B, "dtype": s.dtype,
+    out = {"value": round(value, 3), "unit": UNIT, "ms_per_step": round(t_max / steps, 5), "steps": steps,
+           "warmup": warmup,
+           "config": {"workload": name, "N": N, "D": D, "K": K, "B": B, "dtype": s.dtype,
+                      "iterations_configured": s.iters,
                       "step": "one Lloyd iteration: prepare centroids + assign + update",
-                      "l2": "inputs larger than L2 (X is %d MiB)" % (B * N * D * es >> 20),
-                      "parallelism": "replicas" if world > 1 else "single GPU"},
-           "roofline": roofline, "roofline_update": roofline_update,
-           "gpu_launches": launches,
+                      "l2": "inputs larger than L2 (X is %d MiB)" % (B * N * D * es >> 20)},
+           "roofline": roofline, "roofline_update": roofline_update, "gpu_launches": launches,
            "clocks": clocks.summary(w0, w1)}
-
-    if args.e2e:
-        out["e2e"] = bench_e2e(args, s, w, fk, dev, world)
-    if rank == 0 and world == 1 and args.cpu:
-        import workloads  # noqa: F401
+    if rank == 0 and world == 1 and cpu_budget > 0:
         X64 = X.double().cpu().numpy() if B == 1 else X[0].double().cpu().numpy()
         C64 = w.C0.double().cpu().numpy() if B == 1 else w.C0[0].double().cpu().numpy()
-        v, n, reps, secs, cores = oracle_throughput(X64, C64, s.dtype, N * B, args.cpu_budget)
+        v, n, reps, secs, cores = oracle_throughput(X64, C64, s.dtype, N * B, cpu_budget)
         out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"{reps} x {n} of {N * B} rows against all {K} centroids, one Lloyd "
                                          f"step each ({secs:.1f} s in all), scaled linearly in N"}
+    return out, s, w
+
+
+def bench_gpu(args):
+    import torch
+
+    import distance_argmin_flashassign_b200 as fk
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    head, s, w = measure(args, args.workload, fk, dev, world, rank, args.steps, args.warmup,
+                         args.cpu_budget if args.cpu else 0.0, seed=rank)
+    out = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+           "config": dict(head["config"], parallelism="replicas" if world > 1 else "single GPU"),
+           "roofline": head["roofline"], "roofline_update": head["roofline_update"],
+           "gpu_launches": head["gpu_launches"], "clocks": head["clocks"]}
+    if args.e2e:
+        out["e2e"] = bench_e2e(args, s, w, fk, dev, world)
+    if "cpu_baseline" in head:
+        out["cpu_baseline"] = head["cpu_baseline"]
+    del w
+    torch.cuda.empty_cache()
+    # the other configured workloads, each measured the same way (one GPU)
+    if args.all_workloads and world == 1:
+        others = {}
+        for name in [n for n in ("tiny_f32", "batched_bf16", "zipf_bf16") if n != args.workload]:
+            steps = args.steps if name != "zipf_bf16" else max(3, min(args.steps, 5))
+            res, _, wk = measure(args, name, fk, dev, world, rank, steps, max(3, min(args.warmup, 5)),
+                                 args.other_cpu_budget if args.cpu else 0.0, seed=rank)
+            others[name] = res
+            del wk
+            torch.cuda.empty_cache()
+        if args.ooc_rows_all > 0:
+            others["ooc_f16"] = run_ooc(args, fk, dev, args.ooc_rows_all,
+                                        args.other_cpu_budget if args.cpu else 0.0)
+        out["workloads"] = others
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -384,21 +438,14 @@ def ooc_inputs(rows: int, device):
     return s, Xh, Xh[: s.K].float().clone()  # init = first K rows
 
 
-def bench_ooc(args):
-    """The configured iterations of the out-of-core workload in one
-    fk_lloyd_ooc call: every chunk of X crosses the host link once per
+def run_ooc(args, fk, dev, rows: int, cpu_budget: float):
+    """The configured iterations of the out-of-core workload (at `rows` rows)
+    in one fk_lloyd_ooc call: every chunk of X crosses the host link once per
     iteration on a copy stream while the previous chunk is assigned and
     accumulated.  The host-to-device rate is reported against a plain copy
     of one chunk from the same pinned buffer, timed in this process."""
     import torch
-
-    import distance_argmin_flashassign_b200 as fk
-    rank, world, local = dist_env()
-    if world > 1:
-        raise SystemExit("ooc_f16 runs on one GPU (its pinned host copy of X does not fit once per rank)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    s, Xh, C0 = ooc_inputs(args.ooc_rows, dev)
+    s, Xh, C0 = ooc_inputs(rows, dev)
     N, D, K, chunk, iters = s.N, s.D, s.K, s.chunk_rows, s.iters
     stream = torch.cuda.current_stream(dev)
     # the plain pinned-to-device copy rate of one chunk
@@ -421,7 +468,7 @@ def bench_ooc(args):
     fk.fk_lloyd_ooc(Xh, Ch, 1, chunk, lab_h, cnt_h)  # warm-up: sets up the device ring and workspace
     torch.cuda.synchronize(dev)
     Ch = C0.clone()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     time.sleep(0.3)
     n0 = fk.fk_launch_count()
@@ -437,11 +484,11 @@ def bench_ooc(args):
     value = iters / (ms * 1e-3)
     h2d_gbs = iters * N * D * 2 / (ms * 1e-3) / 1e9
     nchunks = (N + chunk - 1) // chunk
-    out = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1, "steps": iters,
-           "warmup": 1, "ms_per_step": round(ms / iters, 3), "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": s.dtype, "data": "synthetic",
+    out = {"value": round(value, 4), "unit": UNIT, "ms_per_step": round(ms / iters, 3), "steps": iters,
+           "warmup": 1,
            "config": {"workload": "ooc_f16", "N": N, "N_configured": 10 ** 9, "D": D, "K": K, "B": 1,
                       "dtype": s.dtype, "chunk_rows": chunk, "chunks_per_iteration": nchunks,
+                      "iterations_configured": iters,
                       "step": "one Lloyd iteration streamed from pinned host memory (fk_lloyd_ooc, "
                               f"{iters} iterations in one call)",
                       "reduced_N": "the configured 10^9 rows need 256 GB of pinned host memory"},
@@ -452,15 +499,33 @@ def bench_ooc(args):
            "gpu_launches": launches, "clocks": clocks.summary(w0, w1),
            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": N * D * 2 + K * D * 4,
                    "d2h_bytes_per_step": K * D * 4 + K * 4 + (N * 4) // iters}}
-    if args.cpu:
+    if cpu_budget > 0:
         import workloads
         n = min(N, 1 << 16)
         Xs = workloads.rows(s, 0, n, device=dev).cpu()
         v, n_used, reps, secs, cores = oracle_throughput(Xs.double().numpy(), C0.double().numpy(), s.dtype, N,
-                                                         args.cpu_budget)
+                                                         cpu_budget)
         out["cpu_baseline"] = {"value": round(v, 8), "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"{reps} x {n_used} of {N} rows against all {K} centroids, one Lloyd "
                                          f"step each ({secs:.1f} s in all), scaled linearly in N"}
+    del Xh, lab_h
+    return out
+
+
+def bench_ooc(args):
+    import torch
+
+    import distance_argmin_flashassign_b200 as fk
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit("ooc_f16 runs on one GPU (its pinned host copy of X does not fit once per rank)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    r = run_ooc(args, fk, dev, args.ooc_rows, args.cpu_budget if args.cpu else 0.0)
+    out = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": 1, "steps": r["steps"], "warmup": 1,
+           "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f16", "data": "synthetic"}
+    out.update({k: v for k, v in r.items() if k not in ("value", "unit", "ms_per_step", "steps", "warmup")})
     print(json.dumps(out), flush=True)
 
 
@@ -524,6 +589,13 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
+    ap.add_argument("--no-all", dest="all_workloads", action="store_false",
+                    help="measure the headline workload only (skip the other configured workloads)")
+    ap.add_argument("--other-cpu-budget", type=float, default=5.0,
+                    help="seconds of oracle work for each other workload's cpu_baseline")
+    ap.add_argument("--ooc-rows-all", type=int, default=1 << 27,
+                    help="rows of the out-of-core workload in the default line (2^27: 32 GiB pinned, 2 chunks; "
+                         "0 skips it)")
     ap.add_argument("--ooc-rows", type=int, default=1 << 28,
                     help="rows of the out-of-core workload (default 2^28: 64 GiB of pinned fp16, 4 chunks)")
     args = ap.parse_args(argv)
