@@ -68,6 +68,7 @@ def _load():
         "fk_set_wait_timeout_ns": [U64],
         "fk_debug_wait_timeout": [U64, V],
         "fk_release_workspace": [],
+        "fk_debug_inject": [I, I64],
         "fk_version": [],
     }
     for name, args in sig.items():
@@ -87,7 +88,8 @@ lib = _load()
 ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
-             "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_version")
+             "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_debug_inject",
+             "fk_version")
 
 
 def _check(status: int) -> None:
@@ -207,7 +209,8 @@ def fk_update(X, labels, C, counts=None, stream=None):
 
 def fk_update_noalloc(X, labels, C, counts=None, stream=None):
     """fk_update without any device allocation by the library: its scratch is a
-    fixed 32 MiB array inside libfk (about 1.5 M points at D = 128).  For
+    fixed 32 MiB array inside libfk (about 1.55 M points at D = 128 and
+    K = 1,024, 0.41 M at D = 1,024).  For
     callers that cannot let a library allocate (stream capture, a framework
     that owns all device memory, allocation-free loops).  Calls sharing that
     array must not overlap on the GPU."""
@@ -295,6 +298,15 @@ def fk_debug_wait_timeout(ns: int, stream=None) -> int:
 
 def fk_release_workspace() -> None:
     _check(lib.fk_release_workspace())
+
+
+FK_INJECT_NONE, FK_INJECT_CHUNK_COPY, FK_INJECT_SCRATCH_ALLOC = 0, 1, 2
+
+
+def fk_debug_inject(what: int, at: int = -1) -> None:
+    """Arm one host-side test fault (see include/fk.h): FK_INJECT_CHUNK_COPY
+    at chunk copy `at` of the next fk_lloyd_ooc, or FK_INJECT_SCRATCH_ALLOC."""
+    _check(lib.fk_debug_inject(what, at))
 
 
 def fk_version() -> int:

@@ -19,6 +19,16 @@ void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::me
 static std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
 static std::atomic<int> g_assign_path{0};
 
+// Host-side fault injection for tests (fk_debug_inject): one armed fault,
+// disarmed when it fires.  Nothing is done on the device.
+static std::atomic<int> g_inject{0};            // 0 none, 1 chunk copy, 2 scratch allocation
+static std::atomic<long long> g_inject_at{-1};  // chunk copy number within the next out-of-core call
+static bool inject_fires(int what, long long at = -1) {
+  int w = what;
+  if (g_inject.load() != what || (at >= 0 && g_inject_at.load() != at)) return false;
+  return g_inject.compare_exchange_strong(w, 0);
+}
+
 static thread_local fk_status t_last = FK_OK;
 static thread_local std::string t_msg;
 
@@ -85,6 +95,7 @@ static fk_status scratch(DevState &d, cudaStream_t s, size_t need, void **out) {
   std::lock_guard<std::mutex> g(d.mu);
   Scratch &w = d.scratch[s];
   if (w.bytes < need) {
+    if (inject_fires(2)) return fail(FK_ERR_OOM, "scratch allocation failed (injected by fk_debug_inject)");
     if (w.ptr) cudaFreeAsync(w.ptr, s);
     w.ptr = nullptr;
     w.bytes = 0;
@@ -504,6 +515,7 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
     a.acc = acc;
     a.cnt = cnt;
     a.mode = kAccumulate;
+    long long copy_no = 0;  // chunk copies issued by this call
     for (int it = 0; it < iters; ++it) {
       FK_TRY(cudaMemsetAsync(acc, 0, (size_t)K * D * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
       FK_TRY(cudaMemsetAsync(cnt, 0, (size_t)K * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
@@ -514,6 +526,12 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
         const int64_t r0 = c * rows;
         const int nr = (int)((N - r0) < rows ? (N - r0) : rows);
         // copy stream: chunk c into its slot once the compute that last read the slot is done
+        if (inject_fires(1, copy_no)) {
+          rc = fail(FK_ERR_HOST_IO, "host-to-device copy of chunk " + std::to_string(c) + " of iteration " +
+                                        std::to_string(it) + " not issued (injected by fk_debug_inject)");
+          goto done;
+        }
+        ++copy_no;
         FK_TRY(cudaStreamWaitEvent(cs, freed[slot], 0), "cudaStreamWaitEvent", FK_ERR_CUDA);
         FK_TRY(cudaMemcpyAsync(ring[slot], (const char *)X_host + (size_t)r0 * D * es, (size_t)nr * D * es,
                                cudaMemcpyHostToDevice, cs),
@@ -625,6 +643,13 @@ fk_status fk_release_workspace(void) {
   return FK_OK;
 }
 
-int fk_version(void) { return 100; }
+fk_status fk_debug_inject(int what, int64_t at) {
+  if (what < 0 || what > 2 || (what == 1 && at < 0)) return fail(FK_ERR_INVALID_ARG, "what must be 0, 1 or 2");
+  g_inject_at.store(what == 1 ? at : -1);
+  g_inject.store(what);
+  return FK_OK;
+}
+
+int fk_version(void) { return 101; }
 
 }  // extern "C"

@@ -17,17 +17,20 @@
 
 namespace fk {
 
-// 32 MiB: enough for about 1.5 million points at D = 128 (the exact need is
-// computed per call and larger problems are refused).  The array is created
-// on each device when this file's code is first loaded there and stays until
-// the process exits.
+// 32 MiB.  A call needs 16 N + 4 2^b ceil(N / 4096) + 4 (K + 1) +
+// 8 D ceil(N / R) bytes (each term rounded up to 256; b = bits per sort pass,
+// at most 11; R >= 128 sorted positions per gather worker): about 1.55
+// million points at D = 128 and K = 1,024, about 0.41 million at D = 1,024.
+// The need is computed per call and larger problems are refused.  The array
+// is created on each device when this file's code is first loaded there and
+// stays until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 constexpr size_t kNoAllocStatusBytes = 256;  // device status word, then the scratch
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocDevice {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
+  std::mutex mu;
+  bool ready = false;             // set only once the lookup has succeeded
   unsigned char *base = nullptr;  // device address of g_noalloc_scratch
   int sms = 0;
 };
@@ -64,17 +67,30 @@ extern "C" fk_status fk_update_noalloc(const void *X, const int32_t *labels, int
     return record_error(FK_ERR_CUDA, "no usable current CUDA device");
   NoAllocDevice &nd = g_noalloc_dev[dev];
   // Once per device, with that device current: the host-side name of the
-  // array is not a device address, so ask the runtime for the real one.
-  std::call_once(nd.once, [&nd, dev] {
-    void *p = nullptr;
-    nd.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (nd.err == cudaSuccess) nd.err = cudaDeviceGetAttribute(&nd.sms, cudaDevAttrMultiProcessorCount, dev);
-    nd.base = static_cast<unsigned char *>(p);
-  });
-  if (nd.err != cudaSuccess || !nd.base)
-    return record_error(FK_ERR_CUDA, (std::string("cudaGetSymbolAddress(static scratch): ") +
-                                      cudaGetErrorString(nd.err)).c_str());
-  int *status = reinterpret_cast<int *>(nd.base);
+  // array is not a device address, so ask the runtime for the real one.  A
+  // failed lookup is not remembered; the next call tries again.
+  unsigned char *base = nullptr;
+  int sms = 0;
+  {
+    std::lock_guard<std::mutex> g(nd.mu);
+    if (!nd.ready) {
+      void *p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      int n = 0;
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess || !p) {
+        cudaGetLastError();
+        return record_error(FK_ERR_CUDA, (std::string("cudaGetSymbolAddress(static scratch): ") +
+                                          cudaGetErrorString(e)).c_str());
+      }
+      nd.base = static_cast<unsigned char *>(p);
+      nd.sms = n;
+      nd.ready = true;
+    }
+    base = nd.base;
+    sms = nd.sms;
+  }
+  int *status = reinterpret_cast<int *>(base);
   // The status word must start each call at zero; the rest is fully written
   // before it is read.
   if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess)
@@ -90,8 +106,8 @@ extern "C" fk_status fk_update_noalloc(const void *X, const int32_t *labels, int
   a.C = C;
   a.counts = counts;
   a.mode = kMean;
-  const cudaError_t e = launch_update(a, nd.base + kNoAllocStatusBytes, kNoAllocScratchBytes - kNoAllocStatusBytes,
-                                      DevCtl{status, 2000000000ull}, nd.sms, s);
+  const cudaError_t e = launch_update(a, base + kNoAllocStatusBytes, kNoAllocScratchBytes - kNoAllocStatusBytes,
+                                      DevCtl{status, 2000000000ull}, sms, s);
   if (e != cudaSuccess) return record_error(FK_ERR_CUDA, (std::string("update kernels: ") + cudaGetErrorString(e)).c_str());
   return FK_OK;
 }

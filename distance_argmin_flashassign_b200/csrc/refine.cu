@@ -55,7 +55,7 @@ __device__ __forceinline__ void pair_distances(const T *__restrict__ Cb, int D, 
   const bool oka = ka < K, okb = kb < K;
   double sa = 0.0, sb = 0.0;
   if (vec) {
-    constexpr int E = 16 / sizeof(T), NV = 8;
+    constexpr int E = 16 / sizeof(T), NV = sizeof(T) == 4 ? 4 : 8;  // vectors per round
     const uint4 *ra = reinterpret_cast<const uint4 *>(Cb + (size_t)(oka ? ka : 0) * D);
     const uint4 *rb = reinterpret_cast<const uint4 *>(Cb + (size_t)(okb ? kb : 0) * D);
     const int nvec = D / E;
@@ -120,7 +120,7 @@ __device__ __forceinline__ void fold_pair(double da, double db, int ca, int cb, 
 }
 
 template <typename T>
-__global__ void __launch_bounds__(32 * kRefWarps) refine_kernel(const T *__restrict__ X, const T *__restrict__ C,
+__global__ void __launch_bounds__(32 * kRefWarps, 2) refine_kernel(const T *__restrict__ X, const T *__restrict__ C,
                                                                int N, int D, int K, int vec, NearTies t,
                                                                int32_t *__restrict__ labels,
                                                                float *__restrict__ mindist) {
@@ -219,7 +219,7 @@ static cudaError_t launch_t(const void *X, const void *C, int N, int D, int K, N
                             float *mindist, int num_sms, cudaStream_t s) {
   const int vec = ((size_t)D * sizeof(T)) % 16 == 0 && (uintptr_t)C % 16 == 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_sms > 0 ? num_sms : 1);
+  cfg.gridDim = dim3(2 * (num_sms > 0 ? num_sms : 1));
   cfg.blockDim = dim3(32 * kRefWarps);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;

@@ -197,12 +197,15 @@ FK_API fk_status fk_update_batched(const void *X, const int32_t *labels, int B, 
  *   its scratch from a 32 MiB array compiled into the library instead of the
  *   allocation cache; it calls no cudaMalloc, cudaFree or other allocating
  *   routine.
- *   Limits: the scratch needed (about 16 bytes per point plus small tables)
- *   must fit the 32 MiB array -- about 1.5 million points at D = 128; larger
- *   requests return FK_ERR_UNSUPPORTED with the needed size in
- *   fk_last_error_message().
+ *   Limits: the scratch needed, 16 N + 4 2^b ceil(N / 4096) + 4 (K + 1) +
+ *   8 D ceil(N / R) bytes (b: bits per sort pass, at most 11; R >= 128 rows
+ *   per gather worker), must fit the 32 MiB array less 256 bytes -- about
+ *   1.55 million points at D = 128 and K = 1,024, about 0.41 million at
+ *   D = 1,024; larger requests return FK_ERR_UNSUPPORTED with the needed size
+ *   in fk_last_error_message().
  *   Set-up: the first call on each device looks up the array's device address
- *   (no allocation); make that first call before any stream capture.  The
+ *   (no allocation); make that first call before any stream capture.  A
+ *   failed lookup is retried by the next call.  The
  *   array exists on every device where the library's code was loaded and is
  *   held until the process exits.
  *   Sharing: all calls in the process share the one array and it keeps the
@@ -308,7 +311,19 @@ FK_API fk_status fk_debug_wait_timeout(uint64_t ns, fk_stream_t stream);
  * must ensure no fk_* work is still running on that device. */
 FK_API fk_status fk_release_workspace(void);
 
-/* Library version, major * 10000 + minor * 100 + patch. */
+/* Test hook: arm one host-side fault, which fires once and disarms itself.
+ *   what = 1: in the next fk_lloyd_ooc call, chunk copy number `at` (0 = the
+ *             first chunk of the first iteration, counting on across
+ *             iterations) is not issued and the call fails with
+ *             FK_ERR_HOST_IO, as when a copy fails: the call waits for the
+ *             work it already queued on both of its streams and returns;
+ *   what = 2: the next growth of the scratch cache fails as when the device
+ *             is out of memory (FK_ERR_OOM; nothing is queued);
+ *   what = 0: disarm.
+ * Nothing is injected on the device.  Process-wide. */
+FK_API fk_status fk_debug_inject(int what, int64_t at);
+
+/* Library version, major * 10000 + minor * 100 + patch (101: 0.1.1). */
 FK_API int fk_version(void);
 
 #ifdef __cplusplus

@@ -105,3 +105,11 @@ def test_binding_validates_shapes():
         fk.fk_assign(X, torch.zeros(4, 8, dtype=torch.float32))   # C dtype differs from X
     with pytest.raises(ValueError):
         fk.fk_update(X, torch.zeros(9, dtype=torch.int32), torch.zeros(4, 8))
+
+
+def test_debug_inject_arguments():
+    """The fault-injection hook validates its arguments and can be disarmed
+    without a device."""
+    assert fk.lib.fk_debug_inject(3, 0) == fk.FK_ERR_INVALID_ARG
+    assert fk.lib.fk_debug_inject(1, -1) == fk.FK_ERR_INVALID_ARG
+    assert fk.lib.fk_debug_inject(0, -1) == fk.FK_OK
