@@ -341,6 +341,54 @@ def measure(args, name: str, fk, dev, world: int, rank: int, steps: int, warmup:
     return out, s, w
 
 
+def measure_gauss(args, fk, dev, steps: int, warmup: int):
+    """Weighted Gauss sums on the embedding workload's points: G[i] = sum_k
+    w_k exp(-beta |x_i - c_k|^2) over its K = 1,024 initial centroids,
+    positive weights, beta = 2 (the rows are unit vectors).  One call =
+    the bias prep and the tensor-core pass (fp32 accumulation, running
+    log-sum-exp)."""
+    import torch
+    s, w = build_inputs("embed_f16", dev, 0)
+    X, C = w.X, w.C0.to(torch.float16)
+    N, D, K = s.N, s.D, s.K
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    wt = torch.rand(K, generator=g, device=dev) + 0.5
+    G = torch.empty(N, device=dev)
+    logG = torch.empty(N, device=dev)
+    for _ in range(warmup):
+        fk.fk_gauss_sum(X, C, 2.0, w=wt, G=G, logG=logG)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(steps):
+        fk.fk_gauss_sum(X, C, 2.0, w=wt, G=G, logG=logG)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    clocks.stop()
+    fk.fk_sync()
+    ms = e0.elapsed_time(e1) / steps
+    peaks, peak_kind = load_peaks()
+    flops = 2.0 * N * K * D
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"value": round(1e3 / ms, 3), "unit": "calls/s", "ms_per_step": round(ms, 5), "steps": steps,
+            "config": {"workload": "gauss_f16", "N": N, "D": D, "K": K, "dtype": "f16", "beta": 2.0,
+                       "weights": "uniform in [0.5, 1.5)",
+                       "step": "fk_gauss_sum: Gauss-sum bias prep + tensor-core pass with a log-sum-exp epilogue"},
+            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (Gauss-sum epilogue)",
+                         "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tflops / peaks["bf16_tflops"], 4),
+                         "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
+                         "exp2_per_s": round(N * K / (ms * 1e-3), 1), "traffic": None},
+            "clocks": clocks.summary(w0, w1)}
+
+
 def bench_gpu(args):
     import torch
 
@@ -378,6 +426,8 @@ def bench_gpu(args):
             others[name] = res
             del wk
             torch.cuda.empty_cache()
+        others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
+        torch.cuda.empty_cache()
         if args.ooc_rows_all > 0:
             others["ooc_f16"] = run_ooc(args, fk, dev, args.ooc_rows_all,
                                         args.other_cpu_budget if args.cpu else 0.0)

@@ -69,6 +69,7 @@ def _load():
         "fk_debug_wait_timeout": [U64, V],
         "fk_release_workspace": [],
         "fk_debug_inject": [I, I64],
+        "fk_gauss_sum": [V, I64, I, I, V, I, V, I, ctypes.c_float, V, V, V],
         "fk_version": [],
     }
     for name, args in sig.items():
@@ -89,7 +90,7 @@ ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_ass
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_debug_inject",
-             "fk_version")
+             "fk_gauss_sum", "fk_version")
 
 
 def _check(status: int) -> None:
@@ -265,6 +266,23 @@ def fk_lloyd_ooc(X_host, C_host, iters, chunk_rows, labels_host=None, counts_hos
     _check(lib.fk_lloyd_ooc(_ptr(X_host), N, D, _dtype(X_host), _ptr(C_host), K, _ptr(labels_host),
                             _ptr(counts_host), iters, chunk_rows, _stream(stream)))
     return C_host, labels_host, counts_host
+
+
+def fk_gauss_sum(X, C, beta, w=None, signed=False, G=None, logG=None, want=("G", "logG"), stream=None):
+    """Weighted Gauss sums G[i] = sum_k w[k] exp(-beta |x_i - c_k|^2) (C in
+    X's dtype; w fp32 K or None).  Returns (G, logG); pass C = X for Kv."""
+    N, D = X.shape
+    K = C.shape[0]
+    _need(C, "C", X.dtype, (K, D), X.device)
+    if w is not None:
+        _need(w, "w", torch.float32, (K,), X.device)
+    if G is None and "G" in want:
+        G = torch.empty(N, dtype=torch.float32, device=X.device)
+    if logG is None and "logG" in want:
+        logG = torch.empty(N, dtype=torch.float32, device=X.device)
+    _check(lib.fk_gauss_sum(_ptr(X), N, D, _dtype(X), _ptr(C), K, _ptr(w), int(bool(signed)), float(beta), _ptr(G),
+                            _ptr(logG), _stream(stream)))
+    return G, logG
 
 
 def fk_sync(stream=None) -> None:

@@ -166,7 +166,11 @@ struct TcParams {
   int32_t *labels;
   float *mindist;
   const float *xnorm;  // |x|^2 per row (B*N), or null: computed from the X tile
-  NearTies ties;  // where points whose two best scores are too close to order are listed
+  NearTies ties;
+  // Gaussian-sum epilogue: a = 2 beta log2(e); outputs (either may be null)
+  float gs_a;
+  float *gs_log;  // ln of the weighted Gauss sum per row
+  float *gs_val;  // the weighted Gauss sum per row  // where points whose two best scores are too close to order are listed
   DevCtl ctl;
 };
 
@@ -267,7 +271,63 @@ __device__ __forceinline__ void list_near_tie(const NearTies &t, bool valid, flo
   list_append(t, near, (s1 - s3) <= thr, (int)g, other);
 }
 
-template <int KB, bool DX>
+// ------------------------------------------------ Gaussian-sum epilogue ---
+// With the bias of centroid k set to -|c_k|^2/2 + ln(w_k)/(2 beta), the
+// accumulator holds s'_k = <x, c_k> - |c_k|^2/2 + ln(w_k)/(2 beta), and
+// w_k exp(-beta |x - c_k|^2) = exp(-beta |x|^2) exp(2 beta s'_k).  A row keeps
+// the largest s' seen (M) and S = sum of 2^(a (s'_k - M)), a = 2 beta log2(e),
+// rescaled whenever M grows, as the softmax of flash attention does; the sum
+// is exp(-beta |x|^2) 2^(a M) S.
+struct GaussAcc {
+  float M;  // largest score seen
+  float S;  // sum of 2^(a (s' - M)) over the columns seen
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void gauss_fold(GaussAcc &g, const uint32_t (&v)[32], float a) {
+  const float m = max32(v);
+  if (m > g.M) {  // 2^(a (-inf)) = 0 clears S on the first finite chunk
+    g.S *= ex2_approx((g.M - m) * a);
+    g.M = m;
+  }
+  if (g.M == __int_as_float(0xff800000)) return;  // nothing but padding so far
+  const float nb = -g.M * a;
+  float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    t0 += ex2_approx(fmaf(__uint_as_float(v[j]), a, nb));
+    t1 += ex2_approx(fmaf(__uint_as_float(v[j + 1]), a, nb));
+    t2 += ex2_approx(fmaf(__uint_as_float(v[j + 2]), a, nb));
+    t3 += ex2_approx(fmaf(__uint_as_float(v[j + 3]), a, nb));
+  }
+  g.S += (t0 + t1) + (t2 + t3);
+}
+
+// (M, S) of two column halves of a row, merged.
+__device__ __forceinline__ GaussAcc gauss_merge(GaussAcc x, GaussAcc y, float a) {
+  const float M = fmaxf(x.M, y.M);
+  if (M == __int_as_float(0xff800000)) return x;
+  return GaussAcc{M, x.S * ex2_approx((x.M - M) * a) + y.S * ex2_approx((y.M - M) * a)};
+}
+
+// ln and value of exp(-beta |x|^2) 2^(a M) S for a row.
+__device__ __forceinline__ void gauss_store(const TcParams &p, const GaussAcc &g, float xn, size_t o) {
+  const float l2 = lg2_approx(g.S) + p.gs_a * (g.M - 0.5f * xn);  // log2 of the sum
+  if (p.gs_log) p.gs_log[o] = l2 * 0.6931471805599453f;
+  if (p.gs_val) p.gs_val[o] = ex2_approx(l2);
+}
+
+template <int KB, bool DX, bool GS>
 __global__ void __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
                      const __grid_constant__ CUtensorMap bmap, const TcParams p) {
@@ -541,7 +601,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
         const uint32_t xb = (uint32_t)(t % XBUF);
         Best bs;
-        best_init(bs);
+        GaussAcc ga{__int_as_float(0xff800000), 0.f};
+        if constexpr (!GS) best_init(bs);
+        auto fold = [&](const uint32_t (&v)[32], int col) {
+          if constexpr (GS) gauss_fold(ga, v, p.gs_a);
+          else fold_chunk(bs, v, col);
+        };
         // |x|^2 of this thread's row while the unit is multiplied: the X tile
         // has landed once the pair's xfull completes (the leader sees it and
         // tells the peer)
@@ -570,37 +635,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         FK_TMEM_WAIT_LD(va);
         FK_TMEM_WAIT_LD(vb);
         FK_TMEM_LD32(ta + 64, vc);
-        fold_chunk(bs, va, 0);
+        fold(va, 0);
         FK_TMEM_LD32(ta + 96, va);
-        fold_chunk(bs, vb, 32);
+        fold(vb, 32);
         FK_TMEM_WAIT_LD(vc);
         FK_TMEM_WAIT_LD(va);
         FK_TMEM_LD32(ta + 128, vb);
-        fold_chunk(bs, vc, 64);
+        fold(vc, 64);
         FK_TMEM_LD32(ta + 160, vc);
-        fold_chunk(bs, va, 96);
+        fold(va, 96);
         FK_TMEM_WAIT_LD(vb);
         FK_TMEM_WAIT_LD(vc);
         FK_TMEM_LD32(ta + 192, va);
-        fold_chunk(bs, vb, 128);
+        fold(vb, 128);
         FK_TMEM_LD32(ta + 224, vb);
-        fold_chunk(bs, vc, 160);
+        fold(vc, 160);
         FK_TMEM_WAIT_LD(va);
         FK_TMEM_WAIT_LD(vb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) release_acc(a);
-        fold_chunk(bs, va, 192);
-        fold_chunk(bs, vb, 224);
-        const int jm = best_pos(bs);
-        const int bi = jm < 32 ? bs.base + jm : 0;
-        const float s2 = fmaxf(bs.s2, second_in_chunk(bs, jm));
+        fold(va, 192);
+        fold(vb, 224);
         const size_t o_ = (size_t)b * p.N + row;
-        if (row < p.N) {
-          p.labels[o_] = bi;
-          if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, bs.score, xn));
+        if constexpr (GS) {
+          if (row < p.N) gauss_store(p, ga, xn, o_);
+        } else {
+          const int jm = best_pos(bs);
+          const int bi = jm < 32 ? bs.base + jm : 0;
+          const float s2 = fmaxf(bs.s2, second_in_chunk(bs, jm));
+          if (row < p.N) {
+            p.labels[o_] = bi;
+            if (p.mindist) p.mindist[o_] = fmaxf(0.f, fmaf(-2.f, bs.score, xn));
+          }
+          list_near_tie(p.ties, row < p.N, bs.score, s2, bs.s3, xn, o_, bs.base2);
         }
-        list_near_tie(p.ties, row < p.N, bs.score, s2, bs.s3, xn, o_, bs.base2);
         __syncwarp();
         if (lane == 0) mbar_arrive(xempty(xb));
       }
@@ -612,7 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = u / p.upb;
         const int row = (u % p.upb) * kRowsUnit + (int)rank * kRows + r;
         Best bs;
-        best_init(bs);
+        GaussAcc ga{__int_as_float(0xff800000), 0.f};
+        if constexpr (!GS) best_init(bs);
+        auto fold = [&](const uint32_t (&v)[32], int c) {
+          if constexpr (GS) gauss_fold(ga, v, p.gs_a);
+          else fold_chunk(bs, v, c);
+        };
         // this column half's share of |x|^2, or (column half 0) the prepared
         // |x|^2, loaded now and used at the end of the unit
         float xn = 0.f;
@@ -632,22 +706,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           FK_TMEM_WAIT_LD(va);
           FK_TMEM_WAIT_LD(vb);
           FK_TMEM_LD32(ta + 64, vc);
-          fold_chunk(bs, va, col);
+          fold(va, col);
           FK_TMEM_LD32(ta + 96, va);
-          fold_chunk(bs, vb, col + 32);
+          fold(vb, col + 32);
           // chunks 2 and 3: once they are in registers the accumulator is free
           FK_TMEM_WAIT_LD(vc);
           FK_TMEM_WAIT_LD(va);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) release_acc(a);
-          fold_chunk(bs, vc, col + 64);
-          fold_chunk(bs, va, col + 96);
+          fold(vc, col + 64);
+          fold(va, col + 96);
           // half of the row's |x|^2 per column half, while the unit's second
           // tile is multiplied (the first tile's MMAs have read X)
           if (j == 0 && !p.xnorm) xn = x_norm(xb, h * KB * 4, (h + 1) * KB * 4);
         }
         if (!ok) break;
+        if constexpr (GS) {
+          // merge the two column halves: half 1 hands over (M, S) and its
+          // share of |x|^2, half 0 merges and writes
+          if (h == 1) {
+            if (u != u_begin && !(ok = mbar_wait(xchg_empty, xc ^ 1u, abort_flag, p.ctl))) break;
+            xchg[2 * r] = make_float4(ga.M, ga.S, xn, 0.f);
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(xchg_full);
+              mbar_arrive(xempty(xb));
+            }
+          } else {
+            if (!(ok = mbar_wait(xchg_full, xc, abort_flag, p.ctl))) break;
+            const float4 o = xchg[2 * r];
+            const GaussAcc g = gauss_merge(ga, GaussAcc{o.x, o.y}, p.gs_a);
+            if (row < p.N) gauss_store(p, g, xn + o.z, (size_t)b * p.N + row);
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(xchg_empty);
+              mbar_arrive(xempty(xb));
+            }
+          }
+          if (++xb == XBUF) xb = 0;
+          continue;
+        }
         const int jm = best_pos(bs);
         const int bi = jm < 32 ? bs.base + jm : 0;
         const float s2in = second_in_chunk(bs, jm);
@@ -758,7 +857,7 @@ bool tc_aligned(const void *X, const void *C) {
   return ((uintptr_t)X % 16 == 0) && ((uintptr_t)C % 16 == 0);
 }
 
-template <int KB, bool DX>
+template <int KB, bool DX, bool GS>
 static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, TcParams p,
                              int num_sms, cudaStream_t s) {
   static int configured[64] = {};
@@ -772,7 +871,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   {
     std::lock_guard<std::mutex> g(mu);
     if (dev < 64 && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB, DX>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB, DX, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
       if (e != cudaSuccess) return e;
       configured[dev] = 1;
     }
@@ -796,41 +895,70 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB, DX>, xm, cm, bm, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB, DX, GS>, xm, cm, bm, p);
   count_launches(1);
   return e;
+}
+
+// Tensor maps and parameters shared by the arg-min and Gaussian-sum launches.
+static cudaError_t tc_setup(DType dt, const void *X, const void *C, const float *bias, int B, int N, int D, int K,
+                            int Kpad, const float *xnorm, DevCtl ctl, CUtensorMap *xm, CUtensorMap *cm,
+                            CUtensorMap *bm, TcParams *p) {
+  if (!tc_shape_ok(dt, D) || !tc_aligned(X, C) || (uintptr_t)bias % 16 != 0) return cudaErrorNotSupported;
+  if (!encode_3d(xm, dt, X, D, N, B, kRows) || !encode_3d(cm, dt, C, D, K, B, kHalfN) ||
+      !encode_bias_3d(bm, bias, Kpad, B))
+    return cudaErrorNotSupported;
+  *p = TcParams{};
+  p->N = N;
+  p->K = K;
+  p->Kpad = Kpad;
+  p->ntiles = (K + kTileN - 1) / kTileN;
+  p->upb = (N + kRowsUnit - 1) / kRowsUnit;
+  p->total_units = p->upb * B;
+  p->idesc = idesc_f16(dt == kBF16 ? 1 : 0, kRowsUnit, kTileN);
+  p->idesc_bias = idesc_tf32(kRowsUnit, kTileN);
+  p->is_bf16 = dt == kBF16;
+  p->xnorm = xnorm;
+  p->ctl = ctl;
+  if (Kpad < p->ntiles * kTileN) return cudaErrorInvalidValue;  // the bias must cover every tile
+  return cudaSuccess;
+}
+
+template <bool GS>
+static cudaError_t launch_any(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, const TcParams &p,
+                              int D, int num_sms, cudaStream_t s) {
+  if (p.total_units == 0) return cudaSuccess;
+  const int KB = (D + kBlkK - 1) / kBlkK;
+  const bool deep_x = p.ntiles <= 2;
+  if (KB == 1)
+    return deep_x ? launch_kb<1, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false, GS>(xm, cm, bm, p, num_sms, s);
+  return deep_x ? launch_kb<2, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false, GS>(xm, cm, bm, p, num_sms, s);
 }
 
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
                              int D, int K, int Kpad, const float *xnorm, int32_t *labels, float *mindist,
                              NearTies ties, DevCtl ctl, int num_sms, cudaStream_t s) {
-  if (!tc_shape_ok(dt, D) || !tc_aligned(X, C) || (uintptr_t)bias % 16 != 0) return cudaErrorNotSupported;
   CUtensorMap xm, cm, bm;
-  if (!encode_3d(&xm, dt, X, D, N, B, kRows) || !encode_3d(&cm, dt, C, D, K, B, kHalfN) ||
-      !encode_bias_3d(&bm, bias, Kpad, B))
-    return cudaErrorNotSupported;
   TcParams p;
-  p.N = N;
-  p.K = K;
-  p.Kpad = Kpad;
-  p.ntiles = (K + kTileN - 1) / kTileN;
-  p.upb = (N + kRowsUnit - 1) / kRowsUnit;
-  p.total_units = p.upb * B;
-  p.idesc = idesc_f16(dt == kBF16 ? 1 : 0, kRowsUnit, kTileN);
-  p.idesc_bias = idesc_tf32(kRowsUnit, kTileN);
-  p.is_bf16 = dt == kBF16;
+  cudaError_t e = tc_setup(dt, X, C, bias, B, N, D, K, Kpad, xnorm, ctl, &xm, &cm, &bm, &p);
+  if (e != cudaSuccess) return e;
   p.labels = labels;
   p.mindist = mindist;
-  p.xnorm = xnorm;
   p.ties = ties;
-  p.ctl = ctl;
-  p.dyn_bytes = 0;
-  if (p.total_units == 0) return cudaSuccess;
-  if (Kpad < p.ntiles * kTileN) return cudaErrorInvalidValue;  // the bias must cover every tile
-  const int KB = (D + kBlkK - 1) / kBlkK;
-  const bool deep_x = p.ntiles <= 2;
-  if (KB == 1) return deep_x ? launch_kb<1, true>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false>(xm, cm, bm, p, num_sms, s);
-  return deep_x ? launch_kb<2, true>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false>(xm, cm, bm, p, num_sms, s);
+  return launch_any<false>(xm, cm, bm, p, D, num_sms, s);
+}
+
+cudaError_t launch_gauss_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N, int D, int K,
+                            int Kpad, const float *xnorm, float beta, float *log_out, float *val_out, DevCtl ctl,
+                            int num_sms, cudaStream_t s) {
+  CUtensorMap xm, cm, bm;
+  TcParams p;
+  cudaError_t e = tc_setup(dt, X, C, bias, B, N, D, K, Kpad, xnorm, ctl, &xm, &cm, &bm, &p);
+  if (e != cudaSuccess) return e;
+  p.gs_a = 2.f * beta * 1.4426950408889634f;
+  p.gs_log = log_out;
+  p.gs_val = val_out;
+  return launch_any<true>(xm, cm, bm, p, D, num_sms, s);
 }
 
 }  // namespace fk

@@ -568,6 +568,52 @@ done:
   return rc;
 }
 
+fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, const float *w,
+                       int w_signed, float beta, float *G, float *logG, fk_stream_t stream) {
+  fk_status st = check_sizes(1, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (!(beta > 0.f) || !(beta < 3.0e38f)) return fail(FK_ERR_INVALID_ARG, "beta must be a positive finite number");
+  if (w_signed != 0 && w_signed != 1) return fail(FK_ERR_INVALID_ARG, "w_signed must be 0 or 1");
+  if (w_signed && !w) return fail(FK_ERR_INVALID_ARG, "w_signed needs w");
+  if (!G && !logG) return fail(FK_ERR_INVALID_ARG, "G and logG must not both be NULL");
+  if (N == 0) return FK_OK;
+  if (!X || !C) return fail(FK_ERR_INVALID_ARG, "X and C must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const DType t = (DType)dt;
+  const int Kpad = pad_k(K);
+  const size_t cnb = al256(bias_bytes(1, K)), lb = w_signed ? al256((size_t)N * 4) : 0;
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, cnb + 2 * lb, &ws)) != FK_OK) return st;
+  float *bias = (float *)ws;
+  float *lp = w_signed ? (float *)((char *)ws + cnb) : logG;
+  float *lneg = w_signed ? (float *)((char *)ws + cnb + lb) : nullptr;
+  const bool tc = choose_path(t, D) == 1 && tc_aligned(X, C);
+  for (int part = 0; part < (w_signed ? 2 : 1); ++part) {
+    const int sign = part == 0 ? 1 : -1;
+    float *lo = part == 0 ? lp : lneg;
+    float *vo = w_signed ? nullptr : G;
+    cudaError_t e = cudaErrorNotSupported;
+    if (tc) {
+      e = launch_gauss_bias(t, C, K, Kpad, D, w, sign, beta, bias, s);
+      if (e != cudaSuccess) return cuda_fail(e, "Gauss-sum bias kernel");
+      e = launch_gauss_tc(t, X, C, bias, 1, (int)N, D, K, Kpad, nullptr, beta, lo, vo, ctl_of(*d), d->sms, s);
+      if (e != cudaSuccess && e != cudaErrorNotSupported) return cuda_fail(e, "tensor-core Gauss-sum kernel");
+      if (e != cudaSuccess) cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+      e = launch_gauss_simt(t, X, C, (int)N, D, K, w, sign, beta, lo, vo, s);
+      if (e != cudaSuccess) return cuda_fail(e, "CUDA-core Gauss-sum kernel");
+    }
+  }
+  if (w_signed) {
+    cudaError_t e = launch_gauss_combine(lp, lneg, (int)N, logG, G, s);
+    if (e != cudaSuccess) return cuda_fail(e, "Gauss-sum combine kernel");
+  }
+  return FK_OK;
+}
+
 fk_status fk_sync(fk_stream_t stream) {
   DevState *d;
   fk_status st = device_state(&d);

@@ -50,6 +50,22 @@ constexpr float kNearTieTauTc = 9.5367431640625e-7f;
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,
                                int32_t *labels, float *mindist, NearTies ties, cudaStream_t s);
 
+// ---- Gauss sums: sum_k w_k exp(-beta |x_i - c_k|^2) ------------------------
+// Bias of the tensor-core Gauss-sum epilogue for the weights of one sign
+// (prep.cu); one problem.
+cudaError_t launch_gauss_bias(DType dt, const void *C, int K, int Kpad, int D, const float *w, int sign, float beta,
+                              float *bias, cudaStream_t s);
+// Tensor-core pass (assign_tc.cu): ln and/or value of the sum of one sign part.
+cudaError_t launch_gauss_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N, int D, int K,
+                            int Kpad, const float *xnorm, float beta, float *log_out, float *val_out, DevCtl ctl,
+                            int num_sms, cudaStream_t s);
+// CUDA-core pass (gauss.cu) for the other inputs.
+cudaError_t launch_gauss_simt(DType dt, const void *X, const void *C, int N, int D, int K, const float *w, int sign,
+                              float beta, float *log_out, float *val_out, cudaStream_t s);
+// G = e^lp - e^ln and ln G (gauss.cu).
+cudaError_t launch_gauss_combine(const float *lp, const float *ln, int N, float *log_out, float *val_out,
+                                 cudaStream_t s);
+
 // ---- refine.cu: exact re-decision of listed near-ties ---------------------
 cudaError_t launch_refine(DType dt, const void *X, const void *C, int N, int D, int K, NearTies t,
                           int32_t *labels, float *mindist, int num_sms, cudaStream_t s);

@@ -90,6 +90,55 @@ __global__ void __launch_bounds__(256) round_bias_kernel(const float *__restrict
   }
 }
 
+// Bias of the Gaussian-sum epilogue (assign_tc.cu): -|c_k|^2/2 +
+// ln(w_k)/(2 beta) for the part of the weights of one sign (sign > 0: the
+// positive part max(w, 0), sign < 0: the negative part max(-w, 0); w == null
+// means every weight is 1).  A zero weight gets the -inf padding: its column
+// adds nothing.
+template <typename T>
+__global__ void __launch_bounds__(256) gauss_bias_kernel(const T *__restrict__ C, int K, int Kpad, int D,
+                                                         const float *__restrict__ w, int sign, float inv2beta,
+                                                         float *__restrict__ bias) {
+  const int lane = threadIdx.x & 31;
+  for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < Kpad; r += (long long)gridDim.x * 8) {
+    const int j = (int)r;
+    float wj = 0.f;
+    if (j < K) wj = w ? (sign > 0 ? fmaxf(w[j], 0.f) : fmaxf(-w[j], 0.f)) : (sign > 0 ? 1.f : 0.f);
+    if (!(wj > 0.f)) {
+      if (lane == 0) store_bias_padding(bias + r * kBiasTerms);
+      continue;
+    }
+    const T *c = C + (size_t)j * D;
+    float s = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float v = to_f32<T>(c[d]);
+      s = fmaf(v, v, s);
+    }
+    s = warp_sum(s);
+    if (lane == 0) store_bias_terms(bias + r * kBiasTerms, fmaf(logf(wj), inv2beta, -0.5f * s));
+  }
+}
+
+cudaError_t launch_gauss_bias(DType dt, const void *C, int K, int Kpad, int D, const float *w, int sign, float beta,
+                              float *bias, cudaStream_t s) {
+  long long g = (Kpad + 7) / 8;
+  g = g < 1 ? 1 : (g > 4096 ? 4096 : g);
+  const float inv2beta = 0.5f / beta;
+  switch (dt) {
+    case kF32:
+      gauss_bias_kernel<float><<<(int)g, 256, 0, s>>>((const float *)C, K, Kpad, D, w, sign, inv2beta, bias);
+      break;
+    case kF16:
+      gauss_bias_kernel<__half><<<(int)g, 256, 0, s>>>((const __half *)C, K, Kpad, D, w, sign, inv2beta, bias);
+      break;
+    default:
+      gauss_bias_kernel<__nv_bfloat16>
+          <<<(int)g, 256, 0, s>>>((const __nv_bfloat16 *)C, K, Kpad, D, w, sign, inv2beta, bias);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 // |x|^2 of every row of X (fp32 sums of the squares, which are exact for
 // fp16/bf16 inputs): the row norms of the assignment stage, for its near-tie
 // test and its squared distances.  One warp per row, 16-byte loads when rows

@@ -268,6 +268,31 @@ FK_API fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt,
                        fk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fk_gauss_sum -- weighted Gauss sums on the assignment engine.
+ *   "Fast Gauss Sums via Flash Attention", abstract: Gauss kernel sums with
+ *   arbitrary signed weights, evaluated in fused tiles without writing the
+ *   N x K kernel matrix; FlashDiffusion, Figure 4 caption: the same
+ *   matrix-free Gaussian kernel applied to a vector (Kv: pass C = X, w = v).
+ *     G[i] = sum_k w[k] exp(-beta |x_i - c_k|^2)
+ *   computed like the assignment (same tensor-core tiles, inputs in dt,
+ *   fp32 accumulation), with a running log-sum-exp per point instead of the
+ *   arg-min.
+ *   X        device, N x D, dtype dt
+ *   C        device, K x D, dtype dt
+ *   w        device, K fp32, or NULL (every weight 1)
+ *   w_signed 0: the weights are taken as >= 0 (negative entries count as 0),
+ *            one pass over X; 1: any sign, G is the positive part less the
+ *            negative part (two passes)
+ *   beta     > 0
+ *   G        device, N fp32 (out) or NULL; may underflow or overflow in fp32
+ *   logG     device, N fp32 (out) or NULL: ln G (NaN where G <= 0)
+ *   fp16/bf16 with D % 8 == 0, D <= 128 run on tcgen05; other inputs on a
+ *   CUDA-core kernel.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, const float *w,
+                              int w_signed, float beta, float *G, float *logG, fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status, diagnostics and control.
  * ------------------------------------------------------------------------ */
 

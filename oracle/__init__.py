@@ -53,6 +53,8 @@ def _bind(lib):
     lib.oracle_update.restype = ctypes.c_int
     lib.oracle_label_dist.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp, dp]
     lib.oracle_label_dist.restype = None
+    lib.oracle_gauss_sum.argtypes = [dp, ctypes.c_int64, ctypes.c_int, dp, ctypes.c_int, dp, ctypes.c_double, dp, dp]
+    lib.oracle_gauss_sum.restype = None
     lib.oracle_objective.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp]
     lib.oracle_objective.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
@@ -184,6 +186,26 @@ def update(X, labels, K, C_prev, lib=None):
     if rc != 0:
         raise ValueError("oracle_update: label out of range" if rc == -1 else "oracle_update failed")
     return out, counts
+
+
+def gauss_sum(X, C, beta: float, w=None, lib=None):
+    """Weighted Gauss sums G[i] = sum_k w[k] exp(-beta |x_i - c_k|^2) and
+    ln G (NaN where G <= 0), fp64.  Returns (G, logG)."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    N, D = X.shape
+    K = C.shape[0]
+    G = np.zeros(N, np.float64)
+    L = np.zeros(N, np.float64)
+    wp = None
+    if w is not None:
+        w = np.ascontiguousarray(w, dtype=np.float64)
+        wp = _p(w, ctypes.c_double)
+    if N:
+        lib.oracle_gauss_sum(_p(X, ctypes.c_double), N, D, _p(C, ctypes.c_double), K, wp, float(beta),
+                             _p(G, ctypes.c_double), _p(L, ctypes.c_double))
+    return G, L
 
 
 def objective(X, labels, C, lib=None) -> float:

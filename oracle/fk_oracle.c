@@ -116,6 +116,43 @@ void oracle_label_dist(const double *X, const int32_t *labels, int64_t N, int D,
         out[i] = sqdist(X + (size_t)i * (size_t)D, C + (size_t)labels[i] * (size_t)D, D);
 }
 
+/*
+ * Weighted Gauss sums ("Fast Gauss Sums via Flash Attention", abstract):
+ * G[i] = sum_k w[k] exp(-beta |x_i - c_k|^2), w == NULL meaning every weight
+ * is 1, with the direct-difference distance.  The terms of each sign are
+ * summed as a log-sum-exp, P = sum over w > 0, Q = sum over w < 0 of
+ * |w| exp(-beta d): logG[i] = ln P + ln(1 - Q / P) where P > Q (NaN
+ * otherwise) and G[i] = P - Q.  Either output may be NULL.
+ */
+static void lse_add(double *m, double *s, double e) {
+    if (e == -INFINITY) return;
+    if (e > *m) {
+        *s = *s * exp(*m - e) + 1.0;
+        *m = e;
+    } else {
+        *s += exp(e - *m);
+    }
+}
+
+void oracle_gauss_sum(const double *X, int64_t N, int D, const double *C, int K, const double *w, double beta,
+                      double *G, double *logG) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double *x = X + (size_t)i * (size_t)D;
+        double mp = -INFINITY, sp = 0.0, mq = -INFINITY, sq = 0.0;
+        for (int k = 0; k < K; ++k) {
+            const double wk = w ? w[k] : 1.0;
+            if (wk == 0.0) continue;
+            const double e = log(fabs(wk)) - beta * sqdist(x, C + (size_t)k * (size_t)D, D);
+            if (wk > 0.0) lse_add(&mp, &sp, e);
+            else lse_add(&mq, &sq, e);
+        }
+        const double lp = mp + log(sp), lq = mq + log(sq); /* -inf for an empty part */
+        if (G) G[i] = exp(lp) - exp(lq);
+        if (logG) logG[i] = lp > lq ? lp + log1p(-exp(lq - lp)) : NAN;
+    }
+}
+
 /* Lloyd objective J = sum_i |x_i - c_{labels[i]}|^2. */
 double oracle_objective(const double *X, const int32_t *labels, int64_t N, int D,
                         const double *C) {

@@ -29,7 +29,8 @@ def pytest_terminal_summary(terminalreporter):
         return
     tr = terminalreporter
     tr.section("parity statistics (label comparisons against the oracle)")
-    keys = ["N", "mismatch", "near_tie_points", "fp32_ties", "centroid_rel_l2", "slack", "empty_clusters"]
+    keys = ["N", "mismatch", "near_tie_points", "fp32_ties", "centroid_rel_l2", "slack", "empty_clusters",
+            "max_log_err", "tol"]
     for d in STATS:
         tr.write_line(d["case"] + ": " + ", ".join(f"{k}={d[k]:.3g}" if isinstance(d.get(k), float)
                                                    else f"{k}={d[k]}" for k in keys if k in d))

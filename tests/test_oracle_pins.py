@@ -190,6 +190,45 @@ def pin_objective(lib):
     assert oracle.objective(X, lab, C, lib) == pytest.approx(float(mind.sum()), rel=1e-12)
 
 
+def pin_gauss(lib):
+    # one centre, unit weight: the closed form exp(-beta d)
+    X = np.array([[0.0], [1.0], [3.0]])
+    G, L = oracle.gauss_sum(X, np.array([[1.0]]), 0.5, lib=lib)
+    np.testing.assert_allclose(G, np.exp(-0.5 * np.array([1.0, 0.0, 4.0])), rtol=1e-15)
+    np.testing.assert_allclose(L, -0.5 * np.array([1.0, 0.0, 4.0]), rtol=0, atol=1e-15)
+    # hand-worked: x = 0, centres 1 and 2, weights 3 and -1, beta 0.5:
+    # 3 e^-0.5 - e^-2
+    G, L = oracle.gauss_sum(np.zeros((1, 1)), np.array([[1.0], [2.0]]), 0.5, w=np.array([3.0, -1.0]), lib=lib)
+    assert G[0] == pytest.approx(3 * np.exp(-0.5) - np.exp(-2.0), rel=1e-14)
+    assert L[0] == pytest.approx(np.log(3 * np.exp(-0.5) - np.exp(-2.0)), rel=1e-14)
+    # brute force with numpy (explicit differences, exp, weighted sum)
+    rng = np.random.default_rng(15)
+    X = rng.standard_normal((300, 7))
+    C = rng.standard_normal((40, 7))
+    w = rng.uniform(0.1, 2.0, 40)
+    d = ((X[:, None, :] - C[None]) ** 2).sum(-1)
+    G, L = oracle.gauss_sum(X, C, 0.3, w=w, lib=lib)
+    np.testing.assert_allclose(G, (w[None] * np.exp(-0.3 * d)).sum(1), rtol=1e-12)
+    # no weights means unit weights; a large beta is summed in log space
+    G1, _ = oracle.gauss_sum(X, C, 0.3, lib=lib)
+    np.testing.assert_allclose(G1, np.exp(-0.3 * d).sum(1), rtol=1e-12)
+    _, L = oracle.gauss_sum(X, C, 400.0, w=w, lib=lib)
+    e = np.log(w)[None] - 400.0 * d
+    m = e.max(1)
+    np.testing.assert_allclose(L, m + np.log(np.exp(e - m[:, None]).sum(1)), rtol=1e-12)
+    # linearity in the weights; the sign parts combine as G(w+) - G(w-)
+    w2 = rng.uniform(-1.0, 1.0, 40)
+    Ga, _ = oracle.gauss_sum(X, C, 0.3, w=w, lib=lib)
+    Gb, _ = oracle.gauss_sum(X, C, 0.3, w=w2, lib=lib)
+    Gab, _ = oracle.gauss_sum(X, C, 0.3, w=w + w2, lib=lib)
+    np.testing.assert_allclose(Gab, Ga + Gb, rtol=1e-10, atol=1e-13)
+    # symmetry of the Gaussian kernel: u . (K v) = v . (K u) with C = X
+    u, v = rng.standard_normal(300), rng.standard_normal(300)
+    Kv, _ = oracle.gauss_sum(X, X, 0.3, w=v, lib=lib)
+    Ku, _ = oracle.gauss_sum(X, X, 0.3, w=u, lib=lib)
+    assert float(u @ Kv) == pytest.approx(float(v @ Ku), rel=1e-11)
+
+
 def pin_planted(lib):
     rng = np.random.default_rng(8)
     K, D, per = 12, 6, 40
@@ -205,7 +244,7 @@ def pin_planted(lib):
 
 
 PINS = [pin_vq, pin_sklearn_step, pin_hand_1d, pin_ties, pin_k1_mean, pin_prefix_identity,
-        pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_planted]
+        pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_gauss, pin_planted]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -360,6 +399,9 @@ MUTANTS = [
     ("objective drops the last point", "for (int64_t i = 0; i < N; ++i)\n        J +=",
      "for (int64_t i = 0; i + 1 < N; ++i)\n        J +="),
     ("objective not accumulated", "J += sqdist(", "J = sqdist("),
+    ("Gauss exponent sign", "const double e = log(fabs(wk)) - beta *", "const double e = log(fabs(wk)) + beta *"),
+    ("Gauss weight dropped", "const double e = log(fabs(wk)) - beta *", "const double e = 0.0 * log(fabs(wk)) - beta *"),
+    ("Gauss negative part ignored", "if (G) G[i] = exp(lp) - exp(lq);", "if (G) G[i] = exp(lp);"),
     ("last point dropped", "for (int64_t i = 0; i < N; ++i) {\n        int32_t k = labels[i];",
      "for (int64_t i = 0; i + 1 < N; ++i) {\n        int32_t k = labels[i];"),
 ]
