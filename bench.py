@@ -389,6 +389,35 @@ def measure_gauss(args, fk, dev, steps: int, warmup: int):
             "clocks": clocks.summary(w0, w1)}
 
 
+def measure_seed(args, fk, dev, K: int):
+    """k-means++ seeding of the embedding workload (N = 2^20, D = 128, fp16)
+    with K centres: one kernel per centre (fp32-screened D2 update reading X
+    and D2 once, block weight sums, draw in the last block), plus the first
+    round's extra draw kernel.  Timed once after a short warm-up run."""
+    import numpy as np
+    import torch
+    s, w = build_inputs("embed_f16", dev, 0)
+    u = np.random.default_rng(7).random(K)
+    fk.fk_seed_kmeanspp(w.X, 8, u[:8])
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    fk.fk_seed_kmeanspp(w.X, K, u)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    peaks, peak_kind = load_peaks()
+    bytes_per_round = s.N * s.D * 2 + s.N * 8  # X and D2 read (D2 is written only where it drops)
+    gbs = (K - 1) * bytes_per_round / (ms * 1e-3) / 1e9
+    return {"value": round(1e3 / ms, 4), "unit": "seedings/s", "ms_per_step": round(ms, 3), "steps": 1,
+            "config": {"workload": "seed_f16", "N": s.N, "D": s.D, "K": K, "dtype": "f16",
+                       "step": "fk_seed_kmeanspp: K - 1 rounds of D2 update + draw"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"{peak_kind} copy",
+                         "algorithmic_bytes_per_round": bytes_per_round, "traffic": None}}
+
+
 def bench_gpu(args):
     import torch
 
@@ -427,6 +456,7 @@ def bench_gpu(args):
             del wk
             torch.cuda.empty_cache()
         others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
+        others["seed_f16"] = measure_seed(args, fk, dev, 1024)
         torch.cuda.empty_cache()
         if args.ooc_rows_all > 0:
             others["ooc_f16"] = run_ooc(args, fk, dev, args.ooc_rows_all,

@@ -70,6 +70,7 @@ def _load():
         "fk_release_workspace": [],
         "fk_debug_inject": [I, I64],
         "fk_gauss_sum": [V, I64, I, I, V, I, V, I, ctypes.c_float, V, V, V],
+        "fk_seed_kmeanspp": [V, I64, I, I, I, V, V, V],
         "fk_version": [],
     }
     for name, args in sig.items():
@@ -90,7 +91,7 @@ ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_ass
              "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_debug_inject",
-             "fk_gauss_sum", "fk_version")
+             "fk_gauss_sum", "fk_seed_kmeanspp", "fk_version")
 
 
 def _check(status: int) -> None:
@@ -283,6 +284,22 @@ def fk_gauss_sum(X, C, beta, w=None, signed=False, G=None, logG=None, want=("G",
     _check(lib.fk_gauss_sum(_ptr(X), N, D, _dtype(X), _ptr(C), K, _ptr(w), int(bool(signed)), float(beta), _ptr(G),
                             _ptr(logG), _stream(stream)))
     return G, logG
+
+
+def fk_seed_kmeanspp(X, K, u, centers=None, stream=None):
+    """k-means++ seeding: row indices (device int32 K) of K centres of X
+    (N x D) drawn with the caller's uniforms u (K floats in [0, 1))."""
+    import numpy as np
+    N, D = X.shape
+    u = np.ascontiguousarray(np.asarray(u, dtype=np.float64))
+    if u.shape != (K,):
+        raise ValueError("u must hold K draws")
+    if centers is None:
+        centers = torch.empty(K, dtype=torch.int32, device=X.device)
+    _need(centers, "centers", torch.int32, (K,), X.device)
+    _check(lib.fk_seed_kmeanspp(_ptr(X), N, D, _dtype(X), K, ctypes.c_void_p(u.ctypes.data), _ptr(centers),
+                                _stream(stream)))
+    return centers
 
 
 def fk_sync(stream=None) -> None:

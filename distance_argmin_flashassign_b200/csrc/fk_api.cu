@@ -614,6 +614,24 @@ fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, const void 
   return FK_OK;
 }
 
+fk_status fk_seed_kmeanspp(const void *X, int64_t N, int D, fk_dtype dt, int K, const double *u, int32_t *centers,
+                           fk_stream_t stream) {
+  fk_status st = check_sizes(1, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (N < 1) return fail(FK_ERR_INVALID_ARG, "N must be >= 1");
+  if (!X || !u || !centers) return fail(FK_ERR_INVALID_ARG, "X, u and centers must not be NULL");
+  for (int t = 0; t < K; ++t)
+    if (!(u[t] >= 0.0 && u[t] < 1.0)) return fail(FK_ERR_INVALID_ARG, "every u[t] must lie in [0, 1)");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, seed_workspace_bytes(N, D, K), &ws)) != FK_OK) return st;
+  cudaError_t e = launch_seed((DType)dt, X, (int)N, D, K, u, centers, ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "seeding kernels");
+  return read_status(*d, s);
+}
+
 fk_status fk_sync(fk_stream_t stream) {
   DevState *d;
   fk_status st = device_state(&d);

@@ -66,6 +66,12 @@ cudaError_t launch_gauss_simt(DType dt, const void *X, const void *C, int N, int
 cudaError_t launch_gauss_combine(const float *lp, const float *ln, int N, float *log_out, float *val_out,
                                  cudaStream_t s);
 
+// ---- seed.cu: k-means++ seeding ---------------------------------------------
+size_t seed_workspace_bytes(int64_t N, int D, int K);
+// centers[0..K) from the caller's uniforms u_host[0..K) (host memory).
+cudaError_t launch_seed(DType dt, const void *X, int N, int D, int K, const double *u_host, int32_t *centers, void *ws,
+                        cudaStream_t s);
+
 // ---- refine.cu: exact re-decision of listed near-ties ---------------------
 cudaError_t launch_refine(DType dt, const void *X, const void *C, int N, int D, int K, NearTies t,
                           int32_t *labels, float *mindist, int num_sms, cudaStream_t s);

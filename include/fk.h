@@ -293,6 +293,27 @@ FK_API fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, cons
                               int w_signed, float beta, float *G, float *logG, fk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fk_seed_kmeanspp -- k-means++ seeding on the GPU.
+ *   The Japanese Hacker News summary of Flash-KMeans (discussion section):
+ *   seeding (k-means++) is the step before Lloyd's iterations, outside the
+ *   paper's target.  Centre 0 is point floor(u[0] N); centre t is drawn with
+ *   probability proportional to D2(x) = min over the centres so far of
+ *   |x - c|^2, with these reproducible rules: D2 is sum_j (x_j - c_j)^2 in
+ *   fp64, j ascending, each operation rounded; the weights are the integers
+ *   floor(D2 2^s), s the largest exponent with N max D2 2^s < 2^61 for the
+ *   D2 after the first centre; r = floor(u[t] T) for the weights' total T
+ *   (T - 1 if that rounds up to T), and the centre is the first point whose
+ *   running weight exceeds r; with T = 0 it is point floor(u[t] N).
+ *   X        device, N x D, dtype dt, N >= 1
+ *   u        host, K doubles in [0, 1): the draws (the caller's generator)
+ *   centers  device, K int32 (out): row indices of the chosen centres
+ *   Scratch 8 N bytes and a little more.  Two kernels per centre.
+ *   Synchronises `stream`.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_seed_kmeanspp(const void *X, int64_t N, int D, fk_dtype dt, int K, const double *u,
+                                  int32_t *centers, fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status, diagnostics and control.
  * ------------------------------------------------------------------------ */
 

@@ -55,6 +55,8 @@ def _bind(lib):
     lib.oracle_label_dist.restype = None
     lib.oracle_gauss_sum.argtypes = [dp, ctypes.c_int64, ctypes.c_int, dp, ctypes.c_int, dp, ctypes.c_double, dp, dp]
     lib.oracle_gauss_sum.restype = None
+    lib.oracle_kmeanspp.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, ip]
+    lib.oracle_kmeanspp.restype = ctypes.c_int
     lib.oracle_objective.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp]
     lib.oracle_objective.restype = ctypes.c_double
     lib.oracle_num_threads.argtypes = []
@@ -206,6 +208,20 @@ def gauss_sum(X, C, beta: float, w=None, lib=None):
         lib.oracle_gauss_sum(_p(X, ctypes.c_double), N, D, _p(C, ctypes.c_double), K, wp, float(beta),
                              _p(G, ctypes.c_double), _p(L, ctypes.c_double))
     return G, L
+
+
+def kmeanspp(X, K: int, u, lib=None) -> np.ndarray:
+    """k-means++ centre indices (int32 K) drawn with the uniforms u (K in [0, 1))."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    assert u.shape == (K,) and X.shape[0] >= 1
+    out = np.zeros(K, np.int32)
+    rc = lib.oracle_kmeanspp(_p(X, ctypes.c_double), X.shape[0], X.shape[1], K, _p(u, ctypes.c_double),
+                             _p(out, ctypes.c_int32))
+    if rc != 0:
+        raise MemoryError("oracle_kmeanspp")
+    return out
 
 
 def objective(X, labels, C, lib=None) -> float:

@@ -153,6 +153,57 @@ void oracle_gauss_sum(const double *X, int64_t N, int D, const double *C, int K,
     }
 }
 
+/*
+ * k-means++ seeding (Arthur and Vassilvitskii) with reproducible draws:
+ * centre 0 is point floor(u[0] N); centre t is drawn with probability
+ * proportional to D2(x) = min over the chosen centres of |x - c|^2, through
+ * integer weights q = floor(D2 2^s) (s the largest exponent with
+ * N max D2 2^s < 2^61, fixed for the D2 after the first centre): r =
+ * floor(u[t] T) (at most T - 1) for the total T, and the centre is the first
+ * point whose running weight exceeds r; with T = 0, point floor(u[t] N).
+ * Returns 0, or -2 when memory runs out.
+ */
+int oracle_kmeanspp(const double *X, int64_t N, int D, int K, const double *u, int32_t *centers) {
+    double *d2 = (double *)malloc((size_t)N * sizeof(double));
+    if (!d2) return -2;
+    int64_t f = (int64_t)floor(u[0] * (double)N);
+    centers[0] = (int32_t)(f < N ? f : N - 1);
+    int L = 0;
+    while (((int64_t)1 << L) < N) ++L;
+    int s = 0;
+    for (int t = 1; t < K; ++t) {
+        const double *c = X + (size_t)centers[t - 1] * (size_t)D;
+        for (int64_t i = 0; i < N; ++i) {
+            const double d = sqdist(X + (size_t)i * (size_t)D, c, D);
+            d2[i] = (t == 1 || d < d2[i]) ? d : d2[i];
+        }
+        if (t == 1) {
+            double m = 0.0;
+            for (int64_t i = 0; i < N; ++i) m = d2[i] > m ? d2[i] : m;
+            int e = 0;
+            if (m > 0.0) frexp(m, &e);
+            s = m > 0.0 ? 61 - e - L : 0;
+        }
+        int64_t T = 0;
+        for (int64_t i = 0; i < N; ++i) T += (int64_t)floor(ldexp(d2[i], s));
+        if (T == 0) {
+            int64_t k = (int64_t)floor(u[t] * (double)N);
+            centers[t] = (int32_t)(k < N ? k : N - 1);
+            continue;
+        }
+        int64_t r = (int64_t)floor(u[t] * (double)T);
+        if (r >= T) r = T - 1;
+        int64_t run = 0, i = 0;
+        for (; i < N; ++i) {
+            run += (int64_t)floor(ldexp(d2[i], s));
+            if (run > r) break;
+        }
+        centers[t] = (int32_t)i;
+    }
+    free(d2);
+    return 0;
+}
+
 /* Lloyd objective J = sum_i |x_i - c_{labels[i]}|^2. */
 double oracle_objective(const double *X, const int32_t *labels, int64_t N, int D,
                         const double *C) {

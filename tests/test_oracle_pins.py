@@ -229,6 +229,79 @@ def pin_gauss(lib):
     assert float(u @ Kv) == pytest.approx(float(v @ Ku), rel=1e-11)
 
 
+def _kpp_python(X, K, u):
+    """k-means++ with the same reproducible rule, written separately: pure
+    Python sums in dimension order and Python integers for the weights."""
+    import math
+    N, D = X.shape
+    rows = [list(map(float, r)) for r in X]
+    def d2of(a, b):
+        s = 0.0
+        for j in range(D):
+            t = a[j] - b[j]
+            s += t * t
+        return s
+    cen = [min(int(math.floor(u[0] * N)), N - 1)]
+    L = max(0, (N - 1).bit_length())
+    d2 = None
+    s = 0
+    for t in range(1, K):
+        c = rows[cen[-1]]
+        d = [d2of(r, c) for r in rows]
+        d2 = d if d2 is None else [min(a, b) for a, b in zip(d2, d)]
+        if t == 1:
+            m = max(d2)
+            s = 61 - math.frexp(m)[1] - L if m > 0 else 0
+        q = [int(math.floor(math.ldexp(v, s))) for v in d2]
+        T = sum(q)
+        if T == 0:
+            cen.append(min(int(math.floor(u[t] * N)), N - 1))
+            continue
+        r = min(int(math.floor(u[t] * float(T))), T - 1)
+        run = 0
+        for i, qi in enumerate(q):
+            run += qi
+            if run > r:
+                cen.append(i)
+                break
+    return cen
+
+
+def pin_kmeanspp(lib):
+    rng = np.random.default_rng(16)
+    # one centre: point floor(u0 N)
+    X = rng.standard_normal((100, 3))
+    assert oracle.kmeanspp(X, 1, np.array([0.505]), lib).tolist() == [50]
+    # two far clusters: the second centre lies in the other cluster
+    X = np.concatenate([rng.standard_normal((50, 4)), 1000.0 + rng.standard_normal((50, 4))])
+    for u1 in (0.01, 0.3, 0.999):  # cluster A holds about 1e-6 of the weight
+        c = oracle.kmeanspp(X, 2, np.array([0.1, u1]), lib)
+        assert c[0] == 10 and c[1] >= 50
+    # the same rule written separately (Python sums and integers)
+    X = rng.standard_normal((150, 5))
+    u = rng.random(12)
+    assert oracle.kmeanspp(X, 12, u, lib).tolist() == _kpp_python(X, 12, u)
+    # probability proportional to D2: over a fine grid of u1 the second
+    # centre is point i for a share q_i / T of the grid
+    X = rng.standard_normal((40, 2))
+    grid = (np.arange(20000) + 0.5) / 20000
+    counts = np.zeros(40)
+    for u1 in grid:
+        counts[oracle.kmeanspp(X, 2, np.array([0.0, u1]), lib)[1]] += 1
+    d2 = ((X - X[0]) ** 2).sum(1)
+    np.testing.assert_allclose(counts / len(grid), d2 / d2.sum(), atol=2.0 / len(grid))
+    # draws on a weight boundary: points 0, 1, 2 on a line, centre 0 first;
+    # weights 0, 2^56, 2^58 (total 5 * 2^56); u1 = 0.2 gives r = 2^56, which
+    # the running weight of point 1 reaches but does not exceed, so point 2;
+    # u1 = 0 gives r = 0: the first point of positive weight, point 1
+    X = np.array([[0.0], [1.0], [2.0]])
+    assert oracle.kmeanspp(X, 2, np.array([0.0, 0.2]), lib).tolist() == [0, 2]
+    assert oracle.kmeanspp(X, 2, np.array([0.0, 0.0]), lib).tolist() == [0, 1]
+    # every point the same: all weights are zero, centre t is floor(u_t N)
+    X = np.ones((30, 3))
+    assert oracle.kmeanspp(X, 3, np.array([0.2, 0.5, 0.95]), lib).tolist() == [6, 15, 28]
+
+
 def pin_planted(lib):
     rng = np.random.default_rng(8)
     K, D, per = 12, 6, 40
@@ -244,7 +317,8 @@ def pin_planted(lib):
 
 
 PINS = [pin_vq, pin_sklearn_step, pin_hand_1d, pin_ties, pin_k1_mean, pin_prefix_identity,
-        pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_gauss, pin_planted]
+        pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_gauss, pin_kmeanspp,
+        pin_planted]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -402,6 +476,10 @@ MUTANTS = [
     ("Gauss exponent sign", "const double e = log(fabs(wk)) - beta *", "const double e = log(fabs(wk)) + beta *"),
     ("Gauss weight dropped", "const double e = log(fabs(wk)) - beta *", "const double e = 0.0 * log(fabs(wk)) - beta *"),
     ("Gauss negative part ignored", "if (G) G[i] = exp(lp) - exp(lq);", "if (G) G[i] = exp(lp);"),
+    ("seeding weights by distance, not its square",
+     "T += (int64_t)floor(ldexp(d2[i], s));", "T += (int64_t)floor(ldexp(sqrt(d2[i]), s));"),
+    ("seeding without the running minimum", "d2[i] = (t == 1 || d < d2[i]) ? d : d2[i];", "d2[i] = d;"),
+    ("seeding off by one in the draw", "if (run > r) break;", "if (run >= r) break;"),
     ("last point dropped", "for (int64_t i = 0; i < N; ++i) {\n        int32_t k = labels[i];",
      "for (int64_t i = 0; i + 1 < N; ++i) {\n        int32_t k = labels[i];"),
 ]
