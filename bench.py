@@ -213,9 +213,9 @@ def oracle_throughput(X64, C64, dtype: str, N_full: int, budget_s: float):
 
 
 # ------------------------------------------------------------- workloads --
-def build_inputs(name: str, device, seed: int):
+def build_inputs(name: str, device, seed: int, rows: int = 0):
     import workloads
-    s = workloads.spec(name)
+    s = workloads.spec(name, N=rows) if rows else workloads.spec(name)
     w = workloads.make(s, seed=seed, device=device)
     return s, w
 
@@ -234,7 +234,7 @@ def measure(args, name: str, fk, dev, world: int, rank: int, steps: int, warmup:
     ABI, with |x|^2 prepared once (X does not change between iterations).
     Returns the workload's JSON fields and the raw timings."""
     import torch
-    s, w = build_inputs(name, dev, seed)
+    s, w = build_inputs(name, dev, seed, getattr(args, "rows", 0) if name == args.workload else 0)
     dt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[s.dtype]
     X = w.X
     B, N, D, K = s.B, s.N, s.D, s.K
@@ -418,6 +418,9 @@ def measure_seed(args, fk, dev, K: int):
                          "algorithmic_bytes_per_round": bytes_per_round, "traffic": None}}
 
 
+OTHER_WORKLOADS = ("tiny_f32", "batched_bf16", "zipf_bf16", "gauss_f16", "seed_f16", "ooc_f16")
+
+
 def bench_gpu(args):
     import torch
 
@@ -448,17 +451,23 @@ def bench_gpu(args):
     # the other configured workloads, each measured the same way (one GPU)
     if args.all_workloads and world == 1:
         others = {}
-        for name in [n for n in ("tiny_f32", "batched_bf16", "zipf_bf16") if n != args.workload]:
+        pick = set(args.others.split(",")) - {""}
+        unknown = pick - set(OTHER_WORKLOADS)
+        if unknown:
+            raise SystemExit(f"unknown workloads in --others: {sorted(unknown)}")
+        for name in [n for n in ("tiny_f32", "batched_bf16", "zipf_bf16") if n != args.workload and n in pick]:
             steps = args.steps if name != "zipf_bf16" else max(3, min(args.steps, 5))
             res, _, wk = measure(args, name, fk, dev, world, rank, steps, max(3, min(args.warmup, 5)),
                                  args.other_cpu_budget if args.cpu else 0.0, seed=rank)
             others[name] = res
             del wk
             torch.cuda.empty_cache()
-        others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
-        others["seed_f16"] = measure_seed(args, fk, dev, 1024)
+        if "gauss_f16" in pick:
+            others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
+        if "seed_f16" in pick:
+            others["seed_f16"] = measure_seed(args, fk, dev, 1024)
         torch.cuda.empty_cache()
-        if args.ooc_rows_all > 0:
+        if args.ooc_rows_all > 0 and "ooc_f16" in pick:
             others["ooc_f16"] = run_ooc(args, fk, dev, args.ooc_rows_all,
                                         args.other_cpu_budget if args.cpu else 0.0)
         out["workloads"] = others
@@ -671,6 +680,10 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds of oracle work for --impl reference")
     ap.add_argument("--no-all", dest="all_workloads", action="store_false",
                     help="measure the headline workload only (skip the other configured workloads)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="rows per problem of the headline workload (0: as configured); for profiling smaller cases")
+    ap.add_argument("--others", default=",".join(OTHER_WORKLOADS),
+                    help="comma-separated subset of the other workloads to measure after the headline one")
     ap.add_argument("--other-cpu-budget", type=float, default=5.0,
                     help="seconds of oracle work for each other workload's cpu_baseline")
     ap.add_argument("--ooc-rows-all", type=int, default=1 << 27,

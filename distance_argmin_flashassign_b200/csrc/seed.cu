@@ -90,20 +90,42 @@ __device__ __forceinline__ void block_max_bits(unsigned long long b, unsigned lo
 }
 
 struct DrawSmem {
-  long long part[kSeedThreads];  // per-thread range sums, then their exclusive prefix
   long long ws[kSeedThreads / 32];
   long long r;
   int blk, idx, last;
 };
 
+// Exclusive prefix of v over the block; *total gets the block's sum.
+__device__ __forceinline__ long long block_exclusive_scan(long long v, long long *ws, long long *total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ws[w] = incl;
+  __syncthreads();
+  long long before = 0, tot = 0;
+#pragma unroll
+  for (int k = 0; k < kSeedThreads / 32; ++k) {
+    const long long x = ws[k];
+    before += k < w ? x : 0;
+    tot += x;
+  }
+  __syncthreads();  // ws may be reused
+  *total = tot;
+  return before + incl - v;
+}
+
 // Thread 0 has published this block's weight sum in bsum; the block that
 // finishes last draws round t: total T, r, the block whose running weight
 // passes r, the point within it; then centers[t], the chosen row into crow,
 // and the counter reset for the next kernel.  Other blocks return.
-// Thread k of the last block sums the block totals [k P, k P + P); an
-// exclusive scan over the threads places each range, and the thread whose
-// range holds r walks it.  D2 and bsum written by other blocks of the same
-// kernel are read through L2.
+// Thread k of the last block sums the block totals [k P, k P + P) with
+// independent loads; a block-wide exclusive scan places each range and gives
+// T; the one thread whose range holds r walks it.  D2 and bsum written by
+// other blocks of the same kernel are read through L2.
 template <typename T>
 __device__ void draw_if_last(DrawSmem &sm, const T *__restrict__ X, int N, int D, const double *d2,
                              const double *__restrict__ u, int t, const long long *bsum, int s, SeedCtl *ctl,
@@ -115,67 +137,55 @@ __device__ void draw_if_last(DrawSmem &sm, const T *__restrict__ X, int N, int D
   __syncthreads();
   if (!sm.last) return;
   __threadfence();
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nb = (int)gridDim.x, P = (nb + kSeedThreads - 1) / kSeedThreads;
   const int b0 = min(nb, (int)threadIdx.x * P), b1 = min(nb, b0 + P);
   long long mine = 0;
-  for (int b = b0; b < b1; ++b) mine += __ldcg(bsum + b);
-  sm.part[threadIdx.x] = mine;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    long long T = 0;
-    for (int k = 0; k < kSeedThreads; ++k) {
-      const long long v = sm.part[k];
-      sm.part[k] = T;  // exclusive prefix
-      T += v;
-    }
-    if (T == 0) {
+  for (int b = b0; b < b1; b += 8) {
+    long long v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = b + k < b1 ? __ldcg(bsum + b + k) : 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mine += v[k];
+  }
+  long long total;
+  const long long pre = block_exclusive_scan(mine, sm.ws, &total);
+  if (total == 0) {
+    if (threadIdx.x == 0) {
       const long long k = (long long)floor(u[t] * (double)N);
       sm.idx = (int)(k < N ? k : N - 1);
-      sm.blk = -1;
-    } else {
-      long long r = (long long)floor(u[t] * (double)T);
-      if (r >= T) r = T - 1;
-      sm.r = r;
-      sm.blk = -2;  // found below
     }
-  }
-  __syncthreads();
-  if (sm.blk == -2) {
-    const long long r = sm.r, pre = sm.part[threadIdx.x];
+  } else {
+    long long r = (long long)floor(u[t] * (double)total);
+    if (r >= total) r = total - 1;
     if (mine > 0 && pre <= r && r < pre + mine) {
       long long run = pre;
-      int b = b0;
-      for (; b < b1; ++b) {
-        const long long q = __ldcg(bsum + b);
-        if (run + q > r) break;
-        run += q;
+      int hit = b1 - 1;
+      for (int b = b0; b < b1 && hit == b1 - 1; b += 8) {
+        long long v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = b + k < b1 ? __ldcg(bsum + b + k) : 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (hit == b1 - 1 && b + k < b1 - 1) {
+            if (run + v[k] > r) hit = b + k;
+            else run += v[k];
+          }
+        }
       }
-      sm.blk = b;
-      sm.r = r - run;  // rank within block b
-      sm.idx = b * kSeedThreads;
+      sm.blk = hit;
+      sm.r = r - run;  // rank within block hit
+      sm.idx = hit * kSeedThreads;
     }
-  }
-  __syncthreads();
-  if (sm.blk >= 0) {
+    __syncthreads();
     // the first point of block blk whose running weight exceeds the rank
+    const long long rank = sm.r;
     const int j = sm.blk * kSeedThreads + threadIdx.x;
     const long long qj = j < N ? weight_of(__ldcg(d2 + j), s) : 0;
-    long long incl = qj;  // inclusive prefix within the warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane == 31) sm.ws[w] = incl;
-    __syncthreads();
-    long long before = 0;
-    for (int k = 0; k < w; ++k) before += sm.ws[k];
-    incl += before;
-    const long long r = sm.r;
-    if (qj > 0 && incl > r && incl - qj <= r) sm.idx = j;  // the one point whose interval holds r
-    __syncthreads();
+    long long bt;
+    const long long excl = block_exclusive_scan(qj, sm.ws, &bt);
+    if (qj > 0 && excl <= rank && rank < excl + qj) sm.idx = j;  // the one point whose interval holds the rank
   }
+  __syncthreads();
   const int idx = sm.idx;
   if (threadIdx.x == 0) {
     centers[t] = idx;
@@ -229,12 +239,10 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
                                                                   const double *__restrict__ u, int t,
                                                                   int32_t *__restrict__ centers, int Lg) {
   constexpr int G = 32 / L, E = Vec16<T>::E;
-  extern __shared__ __align__(16) double cs[];  // the centre in fp64
   __shared__ DrawSmem sm;
   __shared__ unsigned long long wm[kSeedThreads / 32];
   __shared__ int sh_s;
   const int NV = D / E;
-  for (int j = threadIdx.x; j < D; j += kSeedThreads) cs[j] = (double)crow[j];
   if (threadIdx.x == 0) sh_s = first ? 0 : weight_exponent(ctl, Lg);
   const int lane = threadIdx.x & 31, sub = lane % L, g = lane / L;
   const int r0 = blockIdx.x * kSeedThreads + (threadIdx.x & ~31);
@@ -252,34 +260,42 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
       for (int e = 0; e < E; ++e) cr[m][e] = v < NV ? crow[v * E + e] : 0.f;
     }
     unsigned mine = 0;
-    constexpr int kUnroll = (8 / MV < L ? 8 / MV : L) > 0 ? (8 / MV < L ? 8 / MV : L) : 1;  // <= 8 loads in flight
-#pragma unroll kUnroll
-    for (int i = 0; i < L; ++i) {
-      const int rr = i * G + g, row = r0 + rr;
-      float a = 0.f;
-      if (row < N) {
+    // kU steps at a time: all their loads first, then the sums
+    constexpr int kU = 8 / MV < L ? 8 / MV : L;
+    for (int i0 = 0; i0 < L; i0 += kU) {
+      uint4 q[kU][MV];
+#pragma unroll
+      for (int ii = 0; ii < kU; ++ii) {
+        const int row = r0 + (i0 + ii) * G + g;
 #pragma unroll
         for (int m = 0; m < MV; ++m) {
           const int v = sub + L * m;
-          if (v < NV) {
-            float x[E];
-            Vec16<T>::unpack(__ldg(Xv + (size_t)row * NV + v), x);
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              const float dlt = x[e] - cr[m][e];
-              a = fmaf(dlt, dlt, a);
-            }
-          }
+          q[ii][m] = row < N && v < NV ? __ldg(Xv + (size_t)row * NV + v) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
 #pragma unroll
-      for (int o = L / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      const double o_old = __shfl_sync(0xffffffffu, old, rr);
-      if (sub == 0 && row < N && !screen_rules_out(a, o_old, D)) mine |= 1u << rr;
+      for (int ii = 0; ii < kU; ++ii) {
+        const int rr = (i0 + ii) * G + g, row = r0 + rr;
+        float a = 0.f;
+#pragma unroll
+        for (int m = 0; m < MV; ++m) {
+          float x[E];
+          Vec16<T>::unpack(q[ii][m], x);
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float dlt = x[e] - cr[m][e];  // 0 past the row's end (cr = 0 there)
+            a = fmaf(dlt, dlt, a);
+          }
+        }
+#pragma unroll
+        for (int o = L / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        const double o_old = __shfl_sync(0xffffffffu, old, rr);
+        if (sub == 0 && row < N && !screen_rules_out(a, o_old, D)) mine |= 1u << rr;
+      }
     }
     mask = __reduce_or_sync(0xffffffffu, mine);
   }
-  __syncthreads();  // cs
+  __syncthreads();  // sh_s
   double dn = old;  // this lane's row's D2 after the round
   if (row_l < N && ((mask >> lane) & 1u)) {
     const uint4 *xr = Xv + (size_t)row_l * NV;
@@ -289,7 +305,7 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
       Vec16<T>::unpack(__ldg(xr + v), x);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const double dlt = __dsub_rn((double)x[e], cs[v * E + e]);
+        const double dlt = __dsub_rn((double)x[e], (double)__ldg(crow + v * E + e));
         d = __dadd_rn(d, __dmul_rn(dlt, dlt));
       }
     }
@@ -445,9 +461,8 @@ static cudaError_t run_seed(const void *Xv, int N, int D, int K, const double *u
   const bool vec = (D * sizeof(T)) % 16 == 0 && (uintptr_t)X % 16 == 0;
   if (vec) {
     const RoundKernel<T> k = pick_round_kernel<T>((int)(D * sizeof(T) / 16));
-    const size_t smem = (size_t)D * 8;
     for (int t = 1; t < K; ++t) {
-      k<<<nb, kSeedThreads, smem, s>>>(X, N, D, crow, d2, t == 1, ctl, bsum, u, t, centers, L);
+      k<<<nb, kSeedThreads, 0, s>>>(X, N, D, crow, d2, t == 1, ctl, bsum, u, t, centers, L);
       ++launches;
       if (t == 1) {
         seed_sample_kernel<T><<<nb, kSeedThreads, 0, s>>>(X, N, D, d2, u, t, bsum, ctl, centers, crow, L);
