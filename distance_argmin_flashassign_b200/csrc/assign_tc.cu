@@ -88,10 +88,13 @@ static_assert(kTileN == kCentroidPad, "the bias is padded to whole tiles");
 // fit.  With at most two tiles per unit (small K, e.g. a batch of small
 // problems) a unit's MMAs last less than one X load takes, so the deep-X
 // plan (DX) keeps several units of X in flight and only two tile slots.
+// Rows of up to 128 dimensions keep several X tiles and tile slots in
+// flight; 129 to 256 dimensions (3 or 4 k-blocks) fit two tile slots and two
+// X buffers (one at 4 k-blocks) in the 227 KB of shared memory.
 template <int KB, bool DX> struct TcCfg {
-  static constexpr int XBUF = DX ? (KB == 1 ? 8 : 4) : 2;  // X buffers (units in flight)
+  static constexpr int XBUF = KB >= 4 ? 1 : KB == 3 ? 2 : DX ? (KB == 1 ? 8 : 4) : 2;  // X buffers (units in flight)
   static constexpr int SLOT = KB * kStageBytes + kBiasBytes;  // one tile's centroids and bias terms
-  static constexpr int NSLOT = DX ? (KB == 1 ? 4 : 2) : (KB == 1 ? 9 : 4);  // tile slots in the ring
+  static constexpr int NSLOT = KB >= 3 ? 2 : DX ? (KB == 1 ? 4 : 2) : (KB == 1 ? 9 : 4);  // tile slots in the ring
   static constexpr int X_BYTES = XBUF * KB * kXBytes;
   static constexpr int C_BYTES = NSLOT * SLOT;
   static constexpr int XCHG_BYTES = kRows * 32;    // two float4 per row
@@ -851,7 +854,7 @@ static bool encode_bias_3d(CUtensorMap *m, const float *bias, int Kpad, int B) {
   return r == CUDA_SUCCESS;
 }
 
-bool tc_shape_ok(DType dt, int D) { return dt != kF32 && D % 8 == 0 && D >= 8 && D <= 128; }
+bool tc_shape_ok(DType dt, int D) { return dt != kF32 && D % 8 == 0 && D >= 8 && D <= 256; }
 
 bool tc_aligned(const void *X, const void *C) {
   return ((uintptr_t)X % 16 == 0) && ((uintptr_t)C % 16 == 0);
@@ -932,7 +935,11 @@ static cudaError_t launch_any(const CUtensorMap &xm, const CUtensorMap &cm, cons
   const bool deep_x = p.ntiles <= 2;
   if (KB == 1)
     return deep_x ? launch_kb<1, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false, GS>(xm, cm, bm, p, num_sms, s);
-  return deep_x ? launch_kb<2, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false, GS>(xm, cm, bm, p, num_sms, s);
+  if (KB == 2)
+    return deep_x ? launch_kb<2, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false, GS>(xm, cm, bm, p, num_sms, s);
+  if (KB == 3)
+    return deep_x ? launch_kb<3, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<3, false, GS>(xm, cm, bm, p, num_sms, s);
+  return deep_x ? launch_kb<4, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<4, false, GS>(xm, cm, bm, p, num_sms, s);
 }
 
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,

@@ -205,7 +205,7 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
       cn = cn_ws;
     }
     NearTies tt = ties;
-    tt.tau = kNearTieTauTc;
+    tt.tau = near_tie_tau_tc(D);
     cudaError_t e =
         launch_assign_tc(dt, X, C, cn, B, N, D, K, Kpad, xnorm, labels, mindist, tt, ctl_of(d), d.sms, s);
     if (e == cudaSuccess) {

@@ -41,10 +41,13 @@ cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad
 // magnitude summed (the two distances).
 inline float near_tie_tau_simt(int D) { return (float)(D + 8) * 5.9604644775390625e-8f; }
 // The same for the tensor-core kernel: 16 units of fp32 rounding (2^-20)
-// times a bound on |x|^2 + |c|^2.  Its accumulation order is the hardware's;
-// on the five workloads no point whose score gap exceeded 1.3e-7 (|x|^2 +
-// |c|^2) was misordered, eight times below this width.
+// times a bound on |x|^2 + |c|^2 for rows of up to 128 dimensions, scaled by
+// D / 128 above that (the accumulation error grows with the number of
+// products summed).  Its accumulation order is the hardware's; on the five
+// workloads no point whose score gap exceeded 1.3e-7 (|x|^2 + |c|^2) was
+// misordered, eight times below this width.
 constexpr float kNearTieTauTc = 9.5367431640625e-7f;
+inline float near_tie_tau_tc(int D) { return D > 128 ? kNearTieTauTc * (float)D / 128.f : kNearTieTauTc; }
 
 // ---- assign_simt.cu: CUDA-core assignment (any dtype, any D) --------------
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,

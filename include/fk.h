@@ -23,7 +23,7 @@
  *   dtype      FK_F32, FK_F16 or FK_BF16 tags the element type of X (and of C
  *              where C is given in the input type).  Arithmetic accumulates in
  *              fp32.  fp16/bf16 assignment runs on tcgen05 tensor cores when
- *              D is a multiple of 8 and 8 <= D <= 128; every other case runs on
+ *              D is a multiple of 8 and 8 <= D <= 256; every other case runs on
  *              a CUDA-core kernel (fp32 always does).
  *   Distances  label[i] = argmin_k |x_i - c_k|^2 with ties to the LOWEST k
  *              (the pages are silent on ties).  mindist[i] = that squared
@@ -286,7 +286,7 @@ FK_API fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt,
  *   beta     > 0
  *   G        device, N fp32 (out) or NULL; may underflow or overflow in fp32
  *   logG     device, N fp32 (out) or NULL: ln G (NaN where G <= 0)
- *   fp16/bf16 with D % 8 == 0, D <= 128 run on tcgen05; other inputs on a
+ *   fp16/bf16 with D % 8 == 0, D <= 256 run on tcgen05; other inputs on a
  *   CUDA-core kernel.  Asynchronous on `stream`.
  * ------------------------------------------------------------------------ */
 FK_API fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, const float *w,

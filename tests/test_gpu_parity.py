@@ -29,6 +29,7 @@ def c_in(C0, dtype):
 ASSIGN_SHAPES = [  # (N, D, K): tails in N, D and K; tensor and CUDA-core paths
     (1000, 32, 10), (3001, 128, 300), (257, 8, 1), (5000, 64, 1024), (600, 100, 37),
     (2000, 120, 513), (1000, 16, 700), (4097, 128, 2048), (700, 40, 256), (300, 128, 1),
+    (3000, 192, 300), (2500, 256, 700), (1000, 136, 37), (600, 248, 513),  # 3 and 4 k-blocks on the tensor path
 ]
 
 
