@@ -52,6 +52,7 @@ def _load():
         "fk_update_batched": [V, V, I, I64, I, I, I, V, V, V],
         "fk_update_noalloc": [V, V, I64, I, I, I, V, V, V],
         "fk_lloyd": [V, I64, I, I, V, I, V, V, V, I, V],
+        "fk_lloyd_fused": [V, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_batched": [V, I, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_ooc": [V, I64, I, I, V, I, V, V, I, I64, V],
         "fk_bias_len": [I, I],
@@ -88,7 +89,7 @@ lib = _load()
 
 # names declared in include/fk.h (the C ABI this binding mirrors)
 ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
-             "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
+             "fk_lloyd_fused", "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_debug_inject",
              "fk_gauss_sum", "fk_seed_kmeanspp", "fk_version")
@@ -229,8 +230,10 @@ def fk_update_noalloc(X, labels, C, counts=None, stream=None):
     return C, counts
 
 
-def fk_lloyd(X, C, iters, labels=None, mindist=None, counts=None, want_mindist=False, stream=None):
-    """``iters`` Lloyd iterations; fp32 ``C`` is updated in place.  Synchronous."""
+def fk_lloyd(X, C, iters, labels=None, mindist=None, counts=None, want_mindist=False, stream=None, fused=False):
+    """``iters`` Lloyd iterations; fp32 ``C`` is updated in place.  Synchronous.
+    ``fused``: one pass over X per iteration (fk_lloyd_fused; single problem,
+    centroids that fit in shared memory)."""
     B, N, D, bat = _dims(X)
     K = C.shape[-2]
     lead = (B, N) if bat else (N,)
@@ -242,7 +245,12 @@ def fk_lloyd(X, C, iters, labels=None, mindist=None, counts=None, want_mindist=F
     if counts is None:
         counts = torch.empty(((B, K) if bat else (K,)), dtype=torch.int32, device=X.device)
     _need(labels, "labels", torch.int32, lead, X.device)
-    if bat:
+    if fused:
+        if bat:
+            raise ValueError("the single-pass Lloyd step takes one problem")
+        _check(lib.fk_lloyd_fused(_ptr(X), N, D, _dtype(X), _ptr(C), K, _ptr(labels), _ptr(mindist),
+                                  _ptr(counts), iters, _stream(stream)))
+    elif bat:
         _check(lib.fk_lloyd_batched(_ptr(X), B, N, D, _dtype(X), _ptr(C), K, _ptr(labels), _ptr(mindist),
                                     _ptr(counts), iters, _stream(stream)))
     else:

@@ -439,6 +439,30 @@ fk_status fk_lloyd(const void *X, int64_t N, int D, fk_dtype dt, float *C, int K
   return fk_lloyd_batched(X, 1, N, D, dt, C, K, labels, mindist, counts, iters, stream);
 }
 
+fk_status fk_lloyd_fused(const void *X, int64_t N, int D, fk_dtype dt, float *C, int K, int32_t *labels,
+                         float *mindist, int32_t *counts, int iters, fk_stream_t stream) {
+  fk_status st = check_sizes(1, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (iters < 1) return fail(FK_ERR_INVALID_ARG, "iters must be >= 1");
+  if (!C) return fail(FK_ERR_INVALID_ARG, "C must not be NULL");
+  if (!lloyd_fused_fits(K, D)) return fail(FK_ERR_UNSUPPORTED, "K x D is too large for the single-pass kernel");
+  if (N == 0) return fk_update_batched(X, labels, 1, 0, D, dt, K, C, counts, stream);
+  if (!X || !labels) return fail(FK_ERR_INVALID_ARG, "X and labels must not be NULL");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void *ws = nullptr;
+  if ((st = scratch(*d, s, lloyd_fused_workspace_bytes(K, D, d->sms), &ws)) != FK_OK) return st;
+  const cudaError_t e = launch_lloyd_fused((DType)dt, X, (int)N, D, K, C, labels, mindist, counts, iters, ws,
+                                           ctl_of(*d), d->sms, s);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    return fail(FK_ERR_UNSUPPORTED, "the single-pass kernel cannot be made resident on this device");
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "single-pass Lloyd kernel");
+  return read_status(*d, s);
+}
+
 fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float *C_host, int K,
                        int32_t *labels_host, int32_t *counts_host, int iters, int64_t chunk_rows,
                        fk_stream_t stream) {

@@ -25,6 +25,16 @@ constexpr int kBiasTerms = 8;
 inline size_t bias_bytes(int B, int K) { return (size_t)B * pad_k(K) * kBiasTerms * sizeof(float); }
 inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
 
+// ---- fused.cu: single-pass Lloyd iterations (centroids in shared memory) ---
+// True when K x D fits the single-pass kernel's shared memory.
+bool lloyd_fused_fits(int K, int D);
+size_t lloyd_fused_workspace_bytes(int K, int D, int num_sms);
+// `iters` Lloyd iterations of one problem in one cooperative launch (semantics
+// of fk_lloyd).  cudaErrorNotSupported when the shape does not fit.
+cudaError_t launch_lloyd_fused(DType dt, const void *X, int N, int D, int K, float *C, int32_t *labels,
+                               float *mindist, int32_t *counts, int iters, void *ws, DevCtl ctl, int num_sms,
+                               cudaStream_t s);
+
 // ---- prep.cu: centroid bias (row norms of the assignment stage) -----------
 // bias[b*Kpad + j] = -|C[b][j]|^2 / 2 in fp32 for j < K, -inf for K <= j < Kpad.
 cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, float *bias,

@@ -236,6 +236,24 @@ FK_API fk_status fk_lloyd(const void *X, int64_t N, int D, fk_dtype dt, float *C
                    int32_t *labels, float *mindist, int32_t *counts, int iters,
                    fk_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * fk_lloyd_fused -- fk_lloyd in a single pass over X per iteration, for
+ * problems whose centroids fit in shared memory (K x D about 25,000 values
+ * at most; FK_ERR_UNSUPPORTED otherwise).
+ *   Flash-KMeans abstract: the assignment stage followed by the update
+ *   stage, with chunked-stream overlap; here both stages share one read of
+ *   X: each CTA adds the rows it has just assigned into its own per-cluster
+ *   partial sums, and after a grid-wide barrier the partial sums are combined
+ *   in CTA order and divided.  All iterations run in one cooperative launch.
+ *   Labels are exact as in fk_lloyd (near-ties re-decided in fp64); the
+ *   centroid sums are added in a different (fixed) order than fk_lloyd's, so
+ *   C agrees with it to fp32 rounding, not bit for bit.  Arguments, results
+ *   and errors as fk_lloyd.  Synchronises `stream`.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_lloyd_fused(const void *X, int64_t N, int D, fk_dtype dt, float *C, int K,
+                         int32_t *labels, float *mindist, int32_t *counts, int iters,
+                         fk_stream_t stream);
+
 /* fk_lloyd_batched -- fk_lloyd over B independent problems in one launch per
  * stage (shapes as in fk_assign_batched / fk_update_batched); the iteration
  * follows the Flash-KMeans abstract for each problem. */

@@ -44,7 +44,8 @@ def test_assign_path_choice():
     assert fk.fk_assign_path(1000, 8, torch.float16, 3) == 1
     assert fk.fk_assign_path(1000, 32, torch.float32, 128) == 2   # fp32: CUDA-core kernel
     assert fk.fk_assign_path(1000, 100, torch.float16, 8) == 2    # D not a multiple of 8
-    assert fk.fk_assign_path(1000, 256, torch.float16, 8) == 2    # D above 128
+    assert fk.fk_assign_path(1000, 256, torch.float16, 8) == 1    # up to 256 dimensions on tensor cores
+    assert fk.fk_assign_path(1000, 264, torch.float16, 8) == 2    # D above 256
     assert fk.lib.fk_assign_path(10, 0, 1, 5, 1) == fk.FK_ERR_INVALID_ARG
     assert fk.lib.fk_assign_path(10, 8, 7, 5, 1) == fk.FK_ERR_INVALID_ARG
 
