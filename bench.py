@@ -389,6 +389,52 @@ def measure_gauss(args, fk, dev, steps: int, warmup: int):
             "clocks": clocks.summary(w0, w1)}
 
 
+def measure_fused(args, fk, dev, reps: int):
+    """The tiny workload's configured run (5 Lloyd iterations from the first
+    K rows) through fk_lloyd_fused: one cooperative launch, X read once per
+    iteration.  Timed as `reps` whole runs after 3 untimed ones; the value is
+    iterations per second, comparable with the two-stage tiny_f32 line."""
+    import torch
+    s, w = build_inputs("tiny_f32", dev, 0)
+    X = w.X
+    N, D, K, iters = s.N, s.D, s.K, s.iters
+    C = w.C0.clone()
+    labels = torch.empty(N, dtype=torch.int32, device=dev)
+    counts = torch.empty(K, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        C.copy_(w.C0)
+        fk.fk_lloyd(X, C, iters, labels=labels, counts=counts, fused=True)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(reps):
+        C.copy_(w.C0)
+        fk.fk_lloyd(X, C, iters, labels=labels, counts=counts, fused=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    clocks.stop()
+    ms = e0.elapsed_time(e1) / (reps * iters)
+    props = torch.cuda.get_device_properties(dev)
+    fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_GHZ / 1e3
+    flops = 3.0 * N * K * D  # direct difference: a subtraction and a fused multiply-add per term
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"value": round(1e3 / ms, 3), "unit": UNIT, "ms_per_step": round(ms, 5), "steps": reps * iters,
+            "config": {"workload": "tiny_f32", "N": N, "D": D, "K": K, "dtype": "f32", "iterations": iters,
+                       "step": "fk_lloyd_fused: assignment, exact near-tie re-decision and per-CTA partial sums "
+                               "in one pass over X, grid barrier, combine; all iterations in one launch"},
+            "roofline": {"bound": "alu", "kernel": "lloyd_fused_kernel", "achieved": round(tflops, 3),
+                         "peak": round(fp32_peak, 1), "unit": "TFLOP/s", "frac": round(tflops / fp32_peak, 4),
+                         "peak_kind": "fp32 FMA, derived from unit counts and clock",
+                         "algorithmic_flops_per_iteration": flops, "traffic": None},
+            "clocks": clocks.summary(w0, w1)}
+
+
 def measure_seed(args, fk, dev, K: int):
     """k-means++ seeding of the embedding workload (N = 2^20, D = 128, fp16)
     with K centres: one kernel per centre (fp32-screened D2 update reading X
@@ -418,7 +464,7 @@ def measure_seed(args, fk, dev, K: int):
                          "algorithmic_bytes_per_round": bytes_per_round, "traffic": None}}
 
 
-OTHER_WORKLOADS = ("tiny_f32", "batched_bf16", "zipf_bf16", "gauss_f16", "seed_f16", "ooc_f16")
+OTHER_WORKLOADS = ("tiny_f32", "tiny_f32_fused", "batched_bf16", "zipf_bf16", "gauss_f16", "seed_f16", "ooc_f16")
 
 
 def bench_gpu(args):
@@ -462,6 +508,8 @@ def bench_gpu(args):
             others[name] = res
             del wk
             torch.cuda.empty_cache()
+        if "tiny_f32_fused" in pick:
+            others["tiny_f32_fused"] = measure_fused(args, fk, dev, max(3, min(args.steps, 40)))
         if "gauss_f16" in pick:
             others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
         if "seed_f16" in pick:
