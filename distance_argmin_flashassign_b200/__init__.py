@@ -53,6 +53,7 @@ def _load():
         "fk_update_noalloc": [V, V, I64, I, I, I, V, V, V],
         "fk_lloyd": [V, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_fused": [V, I64, I, I, V, I, V, V, V, I, V],
+        "fk_assign_top2": [V, I64, I, I, V, I, V, V, V, V, V],
         "fk_lloyd_batched": [V, I, I64, I, I, V, I, V, V, V, I, V],
         "fk_lloyd_ooc": [V, I64, I, I, V, I, V, V, I, I64, V],
         "fk_bias_len": [I, I],
@@ -89,7 +90,7 @@ lib = _load()
 
 # names declared in include/fk.h (the C ABI this binding mirrors)
 ABI_NAMES = ("fk_bias_len", "fk_prepare_centroids", "fk_prepare_points", "fk_assign_prepared", "fk_assign", "fk_assign_batched", "fk_update", "fk_update_batched", "fk_update_noalloc", "fk_lloyd",
-             "fk_lloyd_fused", "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
+             "fk_lloyd_fused", "fk_assign_top2", "fk_lloyd_batched", "fk_lloyd_ooc", "fk_sync", "fk_status_string", "fk_get_last_error",
              "fk_last_error_message", "fk_launch_count", "fk_assign_path", "fk_set_assign_path",
              "fk_set_wait_timeout_ns", "fk_debug_wait_timeout", "fk_release_workspace", "fk_debug_inject",
              "fk_gauss_sum", "fk_seed_kmeanspp", "fk_version")
@@ -228,6 +229,26 @@ def fk_update_noalloc(X, labels, C, counts=None, stream=None):
     _check(lib.fk_update_noalloc(_ptr(X), _ptr(labels), N, D, _dtype(X), K, _ptr(C), _ptr(counts),
                                  _stream(stream)))
     return C, counts
+
+
+def fk_assign_top2(X, C, label1=None, label2=None, dist1=None, dist2=None, want_dist=False, stream=None):
+    """The two nearest centroids of every row of X (N x D): (label1, label2,
+    dist1, dist2); C K x D in X's dtype.  Asynchronous on ``stream``."""
+    N, D = X.shape
+    K = C.shape[0]
+    _need(C, "C", X.dtype, (K, D), X.device)
+    if label1 is None:
+        label1 = torch.empty(N, dtype=torch.int32, device=X.device)
+    if label2 is None:
+        label2 = torch.empty(N, dtype=torch.int32, device=X.device)
+    if want_dist:
+        dist1 = torch.empty(N, dtype=torch.float32, device=X.device) if dist1 is None else dist1
+        dist2 = torch.empty(N, dtype=torch.float32, device=X.device) if dist2 is None else dist2
+    _need(label1, "label1", torch.int32, (N,), X.device)
+    _need(label2, "label2", torch.int32, (N,), X.device)
+    _check(lib.fk_assign_top2(_ptr(X), N, D, _dtype(X), _ptr(C), K, _ptr(label1), _ptr(label2), _ptr(dist1),
+                              _ptr(dist2), _stream(stream)))
+    return label1, label2, dist1, dist2
 
 
 def fk_lloyd(X, C, iters, labels=None, mindist=None, counts=None, want_mindist=False, stream=None, fused=False):

@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
   const T *Cb = C + (size_t)b * K * D;
 
   const float inf = __int_as_float(0x7f800000);
+  const int ex = (ties.excl != nullptr && valid) ? ties.excl[(size_t)b * N + row] : -1;  // left out, or -1
   float best = inf, s2 = inf, s3 = inf, s2in = inf;
   int bidx = 0, bbase = 0, base2 = -1;
   for (int k0 = 0; k0 < K; k0 += kSimtTileK) {
@@ -75,7 +76,7 @@ __global__ void __launch_bounds__(kSimtRows) assign_simt_kernel(const T *__restr
     int mi = 0;
 #pragma unroll
     for (int t = 0; t < kSimtTileK; ++t) {
-      const float a = k0 + t < K ? acc[t] : inf;
+      const float a = (k0 + t < K && k0 + t != ex) ? acc[t] : inf;
       if (a < m) {
         m2 = m;
         m = a;

@@ -189,6 +189,15 @@ struct Best {
   uint32_t cand[32];  // the chunk that first reached `score`
 };
 
+// Leave column e of a chunk out (its score becomes -inf), for e in [0, 32).
+__device__ __forceinline__ void mask_col(uint32_t (&v)[32], int e) {
+  if ((unsigned)e < 32u) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i == e) v[i] = 0xff800000u;
+  }
+}
+
 __device__ __forceinline__ void best_init(Best &bs) {
   bs.score = __int_as_float(0xff800000);
   bs.base = 0;
@@ -330,7 +339,7 @@ __device__ __forceinline__ void gauss_store(const TcParams &p, const GaussAcc &g
   if (p.gs_val) p.gs_val[o] = ex2_approx(l2);
 }
 
-template <int KB, bool DX, bool GS>
+template <int KB, bool DX, bool GS, bool EX>
 __global__ void __launch_bounds__(kThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap,
                      const __grid_constant__ CUtensorMap bmap, const TcParams p) {
@@ -606,7 +615,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         Best bs;
         GaussAcc ga{__int_as_float(0xff800000), 0.f};
         if constexpr (!GS) best_init(bs);
-        auto fold = [&](const uint32_t (&v)[32], int col) {
+        int ex = -1;  // the centroid this point leaves out
+        if constexpr (EX) ex = row < p.N ? __ldg(p.ties.excl + (size_t)b * p.N + row) : -1;
+        auto fold = [&](uint32_t (&v)[32], int col) {
+          if constexpr (EX) mask_col(v, ex - col);
           if constexpr (GS) gauss_fold(ga, v, p.gs_a);
           else fold_chunk(bs, v, col);
         };
@@ -686,7 +698,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         Best bs;
         GaussAcc ga{__int_as_float(0xff800000), 0.f};
         if constexpr (!GS) best_init(bs);
-        auto fold = [&](const uint32_t (&v)[32], int c) {
+        int ex = -1;  // the centroid this point leaves out
+        if constexpr (EX) ex = row < p.N ? __ldg(p.ties.excl + (size_t)b * p.N + row) : -1;
+        auto fold = [&](uint32_t (&v)[32], int c) {
+          if constexpr (EX) mask_col(v, ex - c);
           if constexpr (GS) gauss_fold(ga, v, p.gs_a);
           else fold_chunk(bs, v, c);
         };
@@ -860,7 +875,7 @@ bool tc_aligned(const void *X, const void *C) {
   return ((uintptr_t)X % 16 == 0) && ((uintptr_t)C % 16 == 0);
 }
 
-template <int KB, bool DX, bool GS>
+template <int KB, bool DX, bool GS, bool EX>
 static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, TcParams p,
                              int num_sms, cudaStream_t s) {
   static int configured[64] = {};
@@ -874,7 +889,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   {
     std::lock_guard<std::mutex> g(mu);
     if (dev < 64 && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB, DX, GS>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+      cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel<KB, DX, GS, EX>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
       if (e != cudaSuccess) return e;
       configured[dev] = 1;
     }
@@ -898,7 +913,7 @@ static cudaError_t launch_kb(const CUtensorMap &xm, const CUtensorMap &cm, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB, DX, GS>, xm, cm, bm, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, assign_tc_kernel<KB, DX, GS, EX>, xm, cm, bm, p);
   count_launches(1);
   return e;
 }
@@ -927,19 +942,19 @@ static cudaError_t tc_setup(DType dt, const void *X, const void *C, const float 
   return cudaSuccess;
 }
 
-template <bool GS>
+template <bool GS, bool EX>
 static cudaError_t launch_any(const CUtensorMap &xm, const CUtensorMap &cm, const CUtensorMap &bm, const TcParams &p,
                               int D, int num_sms, cudaStream_t s) {
   if (p.total_units == 0) return cudaSuccess;
   const int KB = (D + kBlkK - 1) / kBlkK;
   const bool deep_x = p.ntiles <= 2;
   if (KB == 1)
-    return deep_x ? launch_kb<1, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false, GS>(xm, cm, bm, p, num_sms, s);
+    return deep_x ? launch_kb<1, true, GS, EX>(xm, cm, bm, p, num_sms, s) : launch_kb<1, false, GS, EX>(xm, cm, bm, p, num_sms, s);
   if (KB == 2)
-    return deep_x ? launch_kb<2, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false, GS>(xm, cm, bm, p, num_sms, s);
+    return deep_x ? launch_kb<2, true, GS, EX>(xm, cm, bm, p, num_sms, s) : launch_kb<2, false, GS, EX>(xm, cm, bm, p, num_sms, s);
   if (KB == 3)
-    return deep_x ? launch_kb<3, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<3, false, GS>(xm, cm, bm, p, num_sms, s);
-  return deep_x ? launch_kb<4, true, GS>(xm, cm, bm, p, num_sms, s) : launch_kb<4, false, GS>(xm, cm, bm, p, num_sms, s);
+    return deep_x ? launch_kb<3, true, GS, EX>(xm, cm, bm, p, num_sms, s) : launch_kb<3, false, GS, EX>(xm, cm, bm, p, num_sms, s);
+  return deep_x ? launch_kb<4, true, GS, EX>(xm, cm, bm, p, num_sms, s) : launch_kb<4, false, GS, EX>(xm, cm, bm, p, num_sms, s);
 }
 
 cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N,
@@ -952,7 +967,8 @@ cudaError_t launch_assign_tc(DType dt, const void *X, const void *C, const float
   p.labels = labels;
   p.mindist = mindist;
   p.ties = ties;
-  return launch_any<false>(xm, cm, bm, p, D, num_sms, s);
+  return ties.excl ? launch_any<false, true>(xm, cm, bm, p, D, num_sms, s)
+                    : launch_any<false, false>(xm, cm, bm, p, D, num_sms, s);
 }
 
 cudaError_t launch_gauss_tc(DType dt, const void *X, const void *C, const float *bias, int B, int N, int D, int K,
@@ -965,7 +981,7 @@ cudaError_t launch_gauss_tc(DType dt, const void *X, const void *C, const float 
   p.gs_a = 2.f * beta * 1.4426950408889634f;
   p.gs_log = log_out;
   p.gs_val = val_out;
-  return launch_any<true>(xm, cm, bm, p, D, num_sms, s);
+  return launch_any<true, false>(xm, cm, bm, p, D, num_sms, s);
 }
 
 }  // namespace fk

@@ -158,6 +158,7 @@ static fk_status near_ties(DevState &d, cudaStream_t s, void *list, int64_t rows
   out->done = ctl + 1;
   out->count_hi = ctl + 2;
   out->tau = near_tie_tau_simt(D);
+  out->excl = nullptr;
   return FK_OK;
 }
 
@@ -190,10 +191,11 @@ static int choose_path(DType dt, int D) {
 // kernel then computes it from its X tiles.
 static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
                             const float *cn, float *cn_ws, void *ties_ws, const float *xnorm, int32_t *labels,
-                            float *mindist, cudaStream_t s) {
+                            float *mindist, cudaStream_t s, const int32_t *excl = nullptr) {
   NearTies ties;
   fk_status st = near_ties(d, s, ties_ws, (int64_t)B * N, D, &ties);
   if (st != FK_OK) return st;
+  ties.excl = excl;
   const int path = choose_path(dt, D);
   if (path < 0) return fail(FK_ERR_UNSUPPORTED, "tensor-core path forced for an unsupported shape");
   bool done = false;
@@ -287,6 +289,33 @@ fk_status fk_assign_batched(const void *X, int B, int64_t N, int D, fk_dtype dt,
 fk_status fk_assign(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, int32_t *labels,
                     float *mindist, fk_stream_t stream) {
   return fk_assign_batched(X, 1, N, D, dt, C, K, labels, mindist, stream);
+}
+
+fk_status fk_assign_top2(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, int32_t *label1,
+                         int32_t *label2, float *dist1, float *dist2, fk_stream_t stream) {
+  fk_status st = check_sizes(1, N, D, K, dt);
+  if (st != FK_OK) return st;
+  if (N == 0) return FK_OK;
+  if (!X || !C || !label1 || !label2) return fail(FK_ERR_INVALID_ARG, "X, C, label1 and label2 must not be NULL");
+  if (label1 == label2) return fail(FK_ERR_INVALID_ARG, "label1 and label2 must not alias");
+  DevState *d;
+  if ((st = device_state(&d)) != FK_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  void *ws = nullptr;
+  const size_t cnb = al256(bias_bytes(1, K));
+  if ((st = scratch(*d, s, cnb + ties_bytes(N), &ws)) != FK_OK) return st;
+  const DType t = (DType)dt;
+  // pass 1: the nearest centroid
+  st = run_assign(*d, t, X, 1, (int)N, D, C, K, nullptr, (float *)ws, (char *)ws + cnb, nullptr, label1, dist1, s);
+  if (st != FK_OK) return st;
+  if (K == 1) {  // no second centroid
+    cudaError_t e = cudaMemsetAsync(label2, 0xff, (size_t)N * 4, s);
+    if (e == cudaSuccess && dist2) e = launch_fill_f32(dist2, N, __builtin_huge_valf(), s);
+    return e == cudaSuccess ? FK_OK : cuda_fail(e, "second-label fill");
+  }
+  // pass 2: the nearest of the others (each point leaves its label1 out)
+  return run_assign(*d, t, X, 1, (int)N, D, C, K, nullptr, (float *)ws, (char *)ws + cnb, nullptr, label2, dist2, s,
+                    label1);
 }
 
 int64_t fk_bias_len(int B, int K) {

@@ -40,6 +40,9 @@ struct NearTies {
   int *count_hi;  // entries [cap - *count_hi, cap), the full comparisons
   int cap;
   float tau;
+  // null, or per point a centroid the assignment must leave out (the second
+  // pass of the top-2 assignment excludes each point's nearest centroid)
+  const int32_t *excl;
 };
 
 // Append the listed points of a warp (every lane calls this, `near` and

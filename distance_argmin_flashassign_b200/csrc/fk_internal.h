@@ -41,6 +41,8 @@ cudaError_t launch_bias(DType dt, const void *C, int B, int K, int Kpad, int D, 
                         cudaStream_t s);
 // xnorm[r] = |X[r]|^2 (fp32) for the `rows` rows of D elements of X.
 cudaError_t launch_point_norms(DType dt, const void *X, long long rows, int D, float *xnorm, cudaStream_t s);
+// p[0 .. n) = v.
+cudaError_t launch_fill_f32(float *p, long long n, float v, cudaStream_t s);
 // Cdt = C32 rounded to dt (round-to-nearest-even) and bias of Cdt.
 cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad, int D, void *Cdt,
                               float *bias, cudaStream_t s);

@@ -222,4 +222,18 @@ cudaError_t launch_round_bias(DType dt, const float *C32, int B, int K, int Kpad
   return cudaGetLastError();
 }
 
+__global__ void __launch_bounds__(256) fill_f32_kernel(float *__restrict__ p, long long n, float v) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+cudaError_t launch_fill_f32(float *p, long long n, float v, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  long long g = (n + 255) / 256;
+  if (g > 4096) g = 4096;
+  fill_f32_kernel<<<(int)g, 256, 0, s>>>(p, n, v);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace fk

@@ -13,7 +13,7 @@
 // definition states it, sum over j of (x_j - c_j)^2 in fp64 with j ascending
 // and every operation rounded on its own (no fused multiply-add), takes the
 // first minimum in ascending centroid order, and rewrites the label and the
-// distance.
+// distance.  A point's excluded centroid (NearTies::excl) takes no part.
 //
 // Lane l of a warp owns centroid base + l of each chunk and reads its row
 // with 16-byte loads (all of a round in flight) while x is read from shared
@@ -103,10 +103,15 @@ __device__ __forceinline__ void warp_argmin(double &d, int &k) {
 
 // Fold the two chunks (ca < cb; lanes beyond K hold +inf) into (best, bk):
 // candidates arrive in ascending centroid order, so a later one wins only
-// when strictly closer.
-__device__ __forceinline__ void fold_pair(double da, double db, int ca, int cb, int K, double &best, int &bk) {
+// when strictly closer.  Centroid `ex` (or none, -1) takes no part.
+__device__ __forceinline__ void fold_pair(double da, double db, int ca, int cb, int K, int ex, double &best,
+                                          int &bk) {
   const int lane = threadIdx.x & 31;
-  int ka = ca + lane < K ? ca + lane : 0x7fffffff, kb = cb + lane < K ? cb + lane : 0x7fffffff;
+  const double inf = __longlong_as_double(0x7ff0000000000000ll);
+  int ka = ca + lane < K && ca + lane != ex ? ca + lane : 0x7fffffff;
+  int kb = cb + lane < K && cb + lane != ex ? cb + lane : 0x7fffffff;
+  if (ka == 0x7fffffff) da = inf;
+  if (kb == 0x7fffffff) db = inf;
   warp_argmin(da, ka);
   warp_argmin(db, kb);
   if (ka != 0x7fffffff && (da < best || bk == 0x7fffffff)) {
@@ -155,8 +160,9 @@ __global__ void __launch_bounds__(32 * kRefWarps, 2) refine_kernel(const T *__re
     const int c0 = min(ca, cb), c1 = ca == cb ? K : max(ca, cb);  // c1 = K: nothing to read
     double d0, d1, best = inf;
     int bk = 0x7fffffff;
+    const int ex = t.excl ? t.excl[g] : -1;
     pair_distances<T>(Cb, D, K, c0, c1, xs[w], vec, d0, d1);
-    fold_pair(d0, d1, c0, c1, K, best, bk);
+    fold_pair(d0, d1, c0, c1, K, ex, best, bk);
     if (lane == 0 && bk != 0x7fffffff) {
       labels[g] = bk;
       if (mindist) mindist[g] = (float)best;
@@ -173,11 +179,12 @@ __global__ void __launch_bounds__(32 * kRefWarps, 2) refine_kernel(const T *__re
     __syncwarp();
     double best = inf;
     int bk = 0x7fffffff;
+    const int ex = t.excl ? t.excl[g] : -1;
     for (int pr = w; 2 * pr < nchunks; pr += kRefWarps) {
       const int c0 = 64 * pr, c1 = c0 + 32 < K ? c0 + 32 : K;
       double d0, d1;
       pair_distances<T>(Cb, D, K, c0, c1, xs[w], vec, d0, d1);
-      fold_pair(d0, d1, c0, c1, K, best, bk);
+      fold_pair(d0, d1, c0, c1, K, ex, best, bk);
     }
     if (lane == 0) {
       wbest[w] = best;

@@ -220,6 +220,25 @@ FK_API fk_status fk_update_noalloc(const void *X, const int32_t *labels, int64_t
                                    float *C, int32_t *counts, fk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fk_assign_top2 -- the two nearest centroids of every point (soft /
+ * multi-assignment of border points).
+ *   Flash-GMM abstract (the "similar papers" sidebar of the FlashDiffusion
+ *   page): border vectors are placed in several clusters, without a
+ *   materialised point x cluster matrix.  Here the assignment stage runs
+ *   twice on the fused kernels: label1[i] = argmin_k |x_i - c_k|^2 and
+ *   label2[i] = argmin over k != label1[i], both with ties to the LOWEST k
+ *   and both exact in the sense of fk_assign (near-ties re-decided in fp64).
+ *   dist1 / dist2 (either may be NULL): those squared distances as fk_assign
+ *   reports mindist.  K == 1: label2 = -1 and dist2 = +inf.
+ *   X, C, label1, label2, dist1, dist2 on the device; shapes, dtypes and
+ *   paths as fk_assign; label1 and label2 must not alias.  Asynchronous on
+ *   `stream`.
+ * ------------------------------------------------------------------------ */
+FK_API fk_status fk_assign_top2(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K,
+                                int32_t *label1, int32_t *label2, float *dist1, float *dist2,
+                                fk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * fk_lloyd -- `iters` Lloyd iterations, device resident.
  *   Flash-KMeans abstract: one iteration is the assignment stage followed by
  *   the centroid-update stage; the Japanese Hacker News summary, key points:

@@ -51,6 +51,8 @@ def _bind(lib):
     lib.oracle_assign.restype = None
     lib.oracle_update.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, dp, lp]
     lib.oracle_update.restype = ctypes.c_int
+    lib.oracle_top2.argtypes = [dp, ctypes.c_int64, ctypes.c_int, dp, ctypes.c_int, ip, ip, dp, dp]
+    lib.oracle_top2.restype = None
     lib.oracle_label_dist.argtypes = [dp, ip, ctypes.c_int64, ctypes.c_int, dp, dp]
     lib.oracle_label_dist.restype = None
     lib.oracle_gauss_sum.argtypes = [dp, ctypes.c_int64, ctypes.c_int, dp, ctypes.c_int, dp, ctypes.c_double, dp, dp]
@@ -102,6 +104,25 @@ def assign(X, C, lib=None):
                           _p(labels, ctypes.c_int32), _p(mind, ctypes.c_double),
                           _p(second, ctypes.c_double))
     return labels, mind, second
+
+
+def top2(X, C, lib=None):
+    """The two nearest centroids per row (oracle_top2): (label1, label2, d1, d2),
+    labels int32 (label2 = -1 when K == 1), distances fp64."""
+    lib = lib or load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    N, D = X.shape
+    K = C.shape[0]
+    assert C.shape[1] == D and K >= 1
+    l1 = np.zeros(N, np.int32)
+    l2 = np.zeros(N, np.int32)
+    d1 = np.zeros(N, np.float64)
+    d2 = np.zeros(N, np.float64)
+    if N:
+        lib.oracle_top2(_p(X, ctypes.c_double), N, D, _p(C, ctypes.c_double), K, _p(l1, ctypes.c_int32),
+                        _p(l2, ctypes.c_int32), _p(d1, ctypes.c_double), _p(d2, ctypes.c_double))
+    return l1, l2, d1, d2
 
 
 def label_dist(X, labels, C, lib=None):

@@ -73,6 +73,39 @@ void oracle_assign(const double *X, int64_t N, int D, const double *C, int K,
 }
 
 /*
+ * The two nearest centroids (soft / multi-assignment of border points,
+ * Flash-GMM abstract in the FlashDiffusion page's "similar papers" sidebar):
+ * label1[i] = argmin_k |x_i - c_k|^2, label2[i] = argmin over k != label1[i],
+ * each the first minimum in ascending k; d1, d2 the fp64 distances.
+ * K == 1: label2 = -1, d2 = +inf.
+ */
+void oracle_top2(const double *X, int64_t N, int D, const double *C, int K, int32_t *label1, int32_t *label2,
+                 double *d1, double *d2) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double *x = X + (size_t)i * (size_t)D;
+        double best = INFINITY, runner = INFINITY;
+        int32_t a1 = 0, a2 = -1;
+        for (int k = 0; k < K; ++k) {
+            double d = sqdist(x, C + (size_t)k * (size_t)D, D);
+            if (d < best) {
+                runner = best;
+                a2 = k == 0 ? -1 : a1;
+                best = d;
+                a1 = k;
+            } else if (d < runner || a2 < 0) {
+                runner = d;
+                a2 = k;
+            }
+        }
+        label1[i] = a1;
+        label2[i] = a2;
+        if (d1) d1[i] = best;
+        if (d2) d2[i] = runner;
+    }
+}
+
+/*
  * Centroid-update stage: counts[k] = #{i : labels[i] == k};
  * C_out[k] = (sum of those x_i) / counts[k], or C_prev[k] when counts[k] == 0.
  * Returns 0, or -1 if a label lies outside [0, K).

@@ -316,9 +316,34 @@ def pin_planted(lib):
         np.testing.assert_allclose(Cn[k], X[comp == k].mean(0), rtol=1e-12, atol=1e-12)
 
 
+def pin_top2(lib):
+    """The two nearest centroids: a hand-worked 1-D case with duplicated
+    centroids (ties to the lowest index), K = 1, and brute force on integer
+    data, where every distance is exact and a stable sort of each row's
+    distances gives both labels."""
+    X = np.array([[0.0], [1.0], [2.5], [10.0]])
+    C = np.array([[0.0], [2.0], [3.0], [2.0]])
+    l1, l2, d1, d2 = oracle.top2(X, C, lib)
+    assert l1.tolist() == [0, 0, 1, 2]
+    assert l2.tolist() == [1, 1, 2, 1]
+    assert d1.tolist() == [0.0, 1.0, 0.25, 49.0]
+    assert d2.tolist() == [4.0, 1.0, 0.25, 64.0]
+    l1, l2, d1, d2 = oracle.top2(X, C[:1], lib)
+    assert l1.tolist() == [0] * 4 and l2.tolist() == [-1] * 4 and np.all(np.isinf(d2))
+    rng = np.random.default_rng(21)
+    X = rng.integers(-3, 4, (300, 3)).astype(float)
+    C = rng.integers(-3, 4, (25, 3)).astype(float)
+    dm = ((X[:, None, :] - C[None, :, :]) ** 2).sum(-1)
+    order = np.argsort(dm, axis=1, kind="stable")
+    l1, l2, d1, d2 = oracle.top2(X, C, lib)
+    rows = np.arange(300)
+    assert np.array_equal(l1, order[:, 0]) and np.array_equal(l2, order[:, 1])
+    assert np.array_equal(d1, dm[rows, order[:, 0]]) and np.array_equal(d2, dm[rows, order[:, 1]])
+
+
 PINS = [pin_vq, pin_sklearn_step, pin_hand_1d, pin_ties, pin_k1_mean, pin_prefix_identity,
         pin_permutation, pin_empty_cluster, pin_invariants, pin_objective, pin_gauss, pin_kmeanspp,
-        pin_planted]
+        pin_planted, pin_top2]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -480,6 +505,9 @@ MUTANTS = [
      "T += (int64_t)floor(ldexp(d2[i], s));", "T += (int64_t)floor(ldexp(sqrt(d2[i]), s));"),
     ("seeding without the running minimum", "d2[i] = (t == 1 || d < d2[i]) ? d : d2[i];", "d2[i] = d;"),
     ("seeding off by one in the draw", "if (run > r) break;", "if (run >= r) break;"),
+    ("top-2 runner-up tie to the highest index", "} else if (d < runner || a2 < 0) {",
+     "} else if (d <= runner || a2 < 0) {"),
+    ("top-2 forgets the displaced best", "a2 = k == 0 ? -1 : a1;", "a2 = k;"),
     ("last point dropped", "for (int64_t i = 0; i < N; ++i) {\n        int32_t k = labels[i];",
      "for (int64_t i = 0; i + 1 < N; ++i) {\n        int32_t k = labels[i];"),
 ]
