@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfk.so")
-SOURCES = ["fk_api.cu", "prep.cu", "assign_simt.cu", "assign_tc.cu", "refine.cu", "gauss.cu", "seed.cu", "fused.cu", "update.cu", "noalloc.cu"]
+SOURCES = ["fk_api.cu", "prep.cu", "assign_simt.cu", "assign_tc.cu", "assign_tf32.cu", "refine.cu", "gauss.cu", "seed.cu", "fused.cu", "update.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]

@@ -50,6 +50,10 @@ static fk_status cuda_fail(cudaError_t e, const char *where) {
 struct Scratch {
   void *ptr = nullptr;
   size_t bytes = 0;
+  // the fp32 tensor-core path's split operands (x and c as tf32 hi and lo
+  // parts, |x|^2), apart from the caller's scratch
+  void *aux = nullptr;
+  size_t aux_bytes = 0;
   // near-tie list counters of the assignment kernels (count, done), zeroed
   // once on allocation; the re-decision kernel leaves them zero
   int *ties_ctl = nullptr;
@@ -109,6 +113,27 @@ static fk_status scratch(DevState &d, cudaStream_t s, size_t need, void **out) {
     w.bytes = want;
   }
   *out = w.ptr;
+  return FK_OK;
+}
+
+static fk_status aux_scratch(DevState &d, cudaStream_t s, size_t need, void **out) {
+  std::lock_guard<std::mutex> g(d.mu);
+  Scratch &w = d.scratch[s];
+  if (w.aux_bytes < need) {
+    if (inject_fires(2)) return fail(FK_ERR_OOM, "scratch allocation failed (injected by fk_debug_inject)");
+    if (w.aux) cudaFreeAsync(w.aux, s);
+    w.aux = nullptr;
+    w.aux_bytes = 0;
+    const size_t want = need + need / 4 + 4096;
+    cudaError_t e = cudaMallocAsync(&w.aux, want, s);
+    if (e != cudaSuccess) {
+      w.aux = nullptr;
+      cudaGetLastError();
+      return cuda_fail(e, "cudaMallocAsync(split operands)");
+    }
+    w.aux_bytes = want;
+  }
+  *out = w.aux;
   return FK_OK;
 }
 
@@ -175,12 +200,14 @@ static fk_status check_sizes(int B, int64_t N, int D, int K, fk_dtype dt) {
   return FK_OK;
 }
 
-// 1 = tensor-core kernel, 2 = CUDA-core kernel.
+// 1 = tensor-core kernel (fp16/bf16: kind::f16; fp32: three tf32 passes),
+// 2 = CUDA-core kernel.
+static bool tensor_shape_ok(DType dt, int D) { return dt == kF32 ? tf32_shape_ok(D) : tc_shape_ok(dt, D); }
 static int choose_path(DType dt, int D) {
   const int forced = g_assign_path.load();
   if (forced == 2) return 2;
-  if (forced == 1) return tc_shape_ok(dt, D) ? 1 : -1;
-  return tc_shape_ok(dt, D) ? 1 : 2;
+  if (forced == 1) return tensor_shape_ok(dt, D) ? 1 : -1;
+  return tensor_shape_ok(dt, D) ? 1 : 2;
 }
 
 // Assignment of B problems.  cn (the prepared bias of C: kBiasTerms floats per
@@ -199,7 +226,32 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
   const int path = choose_path(dt, D);
   if (path < 0) return fail(FK_ERR_UNSUPPORTED, "tensor-core path forced for an unsupported shape");
   bool done = false;
-  if (path == 1 && tc_aligned(X, C) && (!cn || (uintptr_t)cn % 16 == 0)) {
+  if (path == 1 && dt == kF32) {
+    // fp32: three tf32 passes (one problem at a time; a batch runs on CUDA cores)
+    if (B == 1 && tc_aligned(X, C) && (!cn || (uintptr_t)cn % 16 == 0)) {
+      const int Kpad = pad_k(K);
+      if (!cn) {
+        cudaError_t e = launch_bias(dt, C, B, K, Kpad, D, cn_ws, s);
+        if (e != cudaSuccess) return cuda_fail(e, "bias kernel");
+        cn = cn_ws;
+      }
+      void *aux = nullptr;
+      if ((st = aux_scratch(d, s, tf32_workspace_bytes(N, D, K), &aux)) != FK_OK) return st;
+      NearTies tt = ties;
+      tt.tau = near_tie_tau_tf32(D);
+      cudaError_t e = launch_assign_tf32((const float *)X, (const float *)C, cn, N, D, K, Kpad, labels, mindist, tt,
+                                         aux, ctl_of(d), d.sms, s);
+      if (e == cudaSuccess) {
+        done = true;
+      } else {
+        if (e != cudaErrorNotSupported) return cuda_fail(e, "tf32 tensor-core assign kernel");
+        cudaGetLastError();
+        if (g_assign_path.load() == 1) return fail(FK_ERR_UNSUPPORTED, "tensor maps could not be encoded");
+      }
+    } else if (g_assign_path.load() == 1) {
+      return fail(FK_ERR_UNSUPPORTED, "the fp32 tensor-core path takes one problem with 16-byte aligned X and C");
+    }
+  } else if (path == 1 && tc_aligned(X, C) && (!cn || (uintptr_t)cn % 16 == 0)) {
     const int Kpad = pad_k(K);
     if (!cn) {
       cudaError_t e = launch_bias(dt, C, B, K, Kpad, D, cn_ws, s);
@@ -450,8 +502,9 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   a.counts = counts;
   a.mode = kMean;
   for (int it = 0; it < iters; ++it) {
-    if (t != kF32) {  // fp32 runs on the CUDA-core kernel, which needs no norms
-      cudaError_t e = launch_round_bias(t, C, B, K, Kpad, D, Cdt, cn, s);
+    {  // the centroids as the assignment reads them (fp16/bf16: rounded) and their bias
+      cudaError_t e = t != kF32 ? launch_round_bias(t, C, B, K, Kpad, D, Cdt, cn, s)
+                                : launch_bias(t, C, B, K, Kpad, D, cn, s);
       if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
     }
     st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, tl, xn, labels, it == iters - 1 ? mindist : nullptr,
@@ -574,6 +627,8 @@ fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt, float 
       FK_TRY(cudaMemsetAsync(cnt, 0, (size_t)K * 8, s), "cudaMemsetAsync", FK_ERR_CUDA);
       if (t != kF32)
         FK_TRY(launch_round_bias(t, c32, 1, K, Kpad, D, cdt, cn, s), "centroid prep kernel", FK_ERR_CUDA);
+      else
+        FK_TRY(launch_bias(t, c32, 1, K, Kpad, D, cn, s), "centroid prep kernel", FK_ERR_CUDA);
       for (int64_t c = 0; c < nchunks; ++c) {
         const int slot = (int)(c & 1);
         const int64_t r0 = c * rows;
@@ -744,6 +799,7 @@ fk_status fk_release_workspace(void) {
   std::lock_guard<std::mutex> g(d->mu);
   for (auto &kv : d->scratch) {
     if (kv.second.ptr) cudaFreeAsync(kv.second.ptr, kv.first);
+    if (kv.second.aux) cudaFreeAsync(kv.second.aux, kv.first);
     if (kv.second.ties_ctl) cudaFreeAsync(kv.second.ties_ctl, kv.first);
   }
   cudaError_t e = cudaDeviceSynchronize();

@@ -25,6 +25,15 @@ constexpr int kBiasTerms = 8;
 inline size_t bias_bytes(int B, int K) { return (size_t)B * pad_k(K) * kBiasTerms * sizeof(float); }
 inline size_t dtype_size(DType dt) { return dt == kF32 ? 4 : 2; }
 
+// ---- assign_tf32.cu: fp32 assignment on tensor cores (three tf32 passes) ---
+bool tf32_shape_ok(int D);
+size_t tf32_workspace_bytes(int64_t N, int D, int K);
+// One problem; ws of tf32_workspace_bytes(N, D, K).  cudaErrorNotSupported when
+// the shape or the tensor maps do not fit.
+cudaError_t launch_assign_tf32(const float *X, const float *C, const float *bias, int N, int D, int K, int Kpad,
+                               int32_t *labels, float *mindist, NearTies ties, void *ws, DevCtl ctl, int num_sms,
+                               cudaStream_t s);
+
 // ---- fused.cu: single-pass Lloyd iterations (centroids in shared memory) ---
 // True when K x D fits the single-pass kernel's shared memory.
 bool lloyd_fused_fits(int K, int D);
@@ -60,6 +69,10 @@ inline float near_tie_tau_simt(int D) { return (float)(D + 8) * 5.96046447753906
 // misordered, eight times below this width.
 constexpr float kNearTieTauTc = 9.5367431640625e-7f;
 inline float near_tie_tau_tc(int D) { return D > 128 ? kNearTieTauTc * (float)D / 128.f : kNearTieTauTc; }
+// The fp32 tensor-core path (three tf32 passes) adds the split's error, below
+// 2.5 2^-21 of sum |x_j c_j| (the dropped lo x lo product and the lo parts'
+// own tf32 rounding): four times the 16-bit path's width.
+inline float near_tie_tau_tf32(int D) { return 4.f * near_tie_tau_tc(D); }
 
 // ---- assign_simt.cu: CUDA-core assignment (any dtype, any D) --------------
 cudaError_t launch_assign_simt(DType dt, const void *X, const void *C, int B, int N, int D, int K,

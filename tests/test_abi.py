@@ -42,7 +42,8 @@ def test_assign_path_choice():
     assert fk.fk_assign_path(1000, 128, torch.float16, 1024) == 1
     assert fk.fk_assign_path(1000, 128, torch.bfloat16, 1024) == 1
     assert fk.fk_assign_path(1000, 8, torch.float16, 3) == 1
-    assert fk.fk_assign_path(1000, 32, torch.float32, 128) == 2   # fp32: CUDA-core kernel
+    assert fk.fk_assign_path(1000, 32, torch.float32, 128) == 1   # fp32: three tf32 passes on tensor cores
+    assert fk.fk_assign_path(1000, 30, torch.float32, 128) == 2   # fp32 rows not whole 16-byte groups
     assert fk.fk_assign_path(1000, 100, torch.float16, 8) == 2    # D not a multiple of 8
     assert fk.fk_assign_path(1000, 256, torch.float16, 8) == 1    # up to 256 dimensions on tensor cores
     assert fk.fk_assign_path(1000, 264, torch.float16, 8) == 2    # D above 256
@@ -56,7 +57,7 @@ def test_forced_path_setting():
         assert fk.fk_assign_path(1000, 128, torch.float16, 1024) == 2
         fk.fk_set_assign_path(1)
         assert fk.fk_assign_path(1000, 128, torch.float16, 1024) == 1
-        assert fk.fk_assign_path(1000, 32, torch.float32, 1024) < 0
+        assert fk.fk_assign_path(1000, 30, torch.float32, 1024) < 0
     finally:
         fk.fk_set_assign_path(0)
     with pytest.raises(fk.FKError):

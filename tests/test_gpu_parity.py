@@ -52,8 +52,6 @@ def test_near_ties_are_decided_exactly(dtype, path):
     points have two candidates whose distances differ by less than the fp32
     error of the kernels' scores.  The listed near-ties are re-decided in
     fp64 exactly as the oracle computes, so every label equals the oracle's."""
-    if dtype == "f32" and path == 1:
-        pytest.skip("fp32 runs on the CUDA-core kernel only")
     g = torch.Generator().manual_seed(21)
     N, D, half = 6000, 128, 300
     base = (torch.randn(half, D, generator=g) * 2.0 + 3.0).to(TORCH_DT[dtype])
@@ -118,7 +116,7 @@ def test_prepared_points_and_assign(dtype):
     check_labels(f64(X), f64(C_dt), l1, dtype, gpu_mindist=m1, exact=True, case=f"prepared points {dtype}")
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
 def test_tensor_and_cuda_core_paths_agree(dtype):
     X, C0 = mixture(6000, 128, 777, dtype, seed=3)
     Xd, Cd = X.to(DEV), c_in(C0, dtype).to(DEV)
@@ -142,8 +140,6 @@ def test_integer_inputs_bit_exact_with_ties(dtype, path, K):
     lowest-index tie-breaks on duplicated centroids) and mindist are exact.
     K = 200 fits one 256-centroid tile (each point's whole row of scores is
     read by one warp); K = 300 spans two."""
-    if dtype == "f32" and path == 1:
-        pytest.skip("fp32 runs on the CUDA-core kernel only")
     g = torch.Generator().manual_seed(5)
     N, D = 3000, 64
     third = K // 3
