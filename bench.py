@@ -214,8 +214,13 @@ def oracle_throughput(X64, C64, dtype: str, N_full: int, budget_s: float):
 
 # ------------------------------------------------------------- workloads --
 def build_inputs(name: str, device, seed: int, rows: int = 0):
+    """The configured workload `name`; "embed_f32" is the embedding recipe in
+    fp32 (the fp32 tensor-core case, not a configured workload)."""
     import workloads
-    s = workloads.spec(name, N=rows) if rows else workloads.spec(name)
+    base, over = (("embed_f16", {"dtype": "f32"}) if name == "embed_f32" else (name, {}))
+    if rows:
+        over["N"] = rows
+    s = workloads.spec(base, **over)
     w = workloads.make(s, seed=seed, device=device)
     return s, w
 
@@ -223,6 +228,7 @@ def build_inputs(name: str, device, seed: int, rows: int = 0):
 # Spec peaks of a B200 (the stricter denominators, reported next to the
 # measured ones): dense fp16/bf16 tensor throughput and HBM3e bandwidth.
 SPEC_P16_TFLOPS = 2250.0
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 / bf16 rate
 SPEC_HBM_GBS = 8000.0
 
 
@@ -295,8 +301,22 @@ def measure(args, name: str, fk, dev, world: int, rank: int, steps: int, warmup:
     tflops = flops / (t_assign * 1e-3) / 1e12
     gbs = upd_bytes / (t_update * 1e-3) / 1e9
     stage = "assignment stage: assign kernel + exact near-tie re-decision kernel"
-    if s.dtype == "f32":
-        # fp32 runs on the CUDA-core kernel: bound by the FP32 FMA pipes, whose
+    if s.dtype == "f32" and fk.fk_assign_path(N, D, torch.float32, K) == 1:
+        # fp32 on the tensor cores as three tf32 passes: the tensor work is 3 x
+        # 2NKD, against the tf32 dense peak (the measured bf16 burst peak times
+        # the nominal tf32 / bf16 dense ratio, 1.1 / 2.25)
+        tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
+        work = 3.0 * flops
+        tf = work / (t_assign * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "assign_tf32_kernel (three tf32 passes)",
+                    "stage": stage + " + the hi/lo split of X and C", "achieved": round(tf, 2),
+                    "peak": round(tf32_peak, 1), "unit": "TFLOP/s", "frac": round(tf / tf32_peak, 4),
+                    "peak_kind": f"{peak_kind} bf16 burst x 1.1/2.25 (nominal tf32/bf16 dense ratio)",
+                    "fp32_equivalent_tflops": round(tflops, 2), "traffic": None,
+                    "ms_per_launch": round(t_assign, 5), "algorithmic_flops_per_launch": flops,
+                    "tensor_flops_per_launch": work}
+    elif s.dtype == "f32":
+        # fp32 on the CUDA-core kernel: bound by the FP32 FMA pipes, whose
         # peak is derived from the unit counts and the maximum SM clock
         props = torch.cuda.get_device_properties(dev)
         fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * SM_MAX_GHZ / 1e3
@@ -464,7 +484,8 @@ def measure_seed(args, fk, dev, K: int):
                          "algorithmic_bytes_per_round": bytes_per_round, "traffic": None}}
 
 
-OTHER_WORKLOADS = ("tiny_f32", "tiny_f32_fused", "batched_bf16", "zipf_bf16", "gauss_f16", "seed_f16", "ooc_f16")
+OTHER_WORKLOADS = ("tiny_f32", "tiny_f32_fused", "batched_bf16", "zipf_bf16", "embed_f32", "gauss_f16", "seed_f16",
+                   "ooc_f16")
 
 
 def bench_gpu(args):
@@ -501,8 +522,8 @@ def bench_gpu(args):
         unknown = pick - set(OTHER_WORKLOADS)
         if unknown:
             raise SystemExit(f"unknown workloads in --others: {sorted(unknown)}")
-        for name in [n for n in ("tiny_f32", "batched_bf16", "zipf_bf16") if n != args.workload and n in pick]:
-            steps = args.steps if name != "zipf_bf16" else max(3, min(args.steps, 5))
+        for name in [n for n in ("tiny_f32", "batched_bf16", "zipf_bf16", "embed_f32") if n != args.workload and n in pick]:
+            steps = args.steps if name not in ("zipf_bf16", "embed_f32") else max(3, min(args.steps, 20 if name == "embed_f32" else 5))
             res, _, wk = measure(args, name, fk, dev, world, rank, steps, max(3, min(args.warmup, 5)),
                                  args.other_cpu_budget if args.cpu else 0.0, seed=rank)
             others[name] = res
