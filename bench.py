@@ -172,7 +172,7 @@ class ClockSampler:
 # --------------------------------------------------------- profile data --
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("assign_tc.cu", "fk_common.cuh"):
+    for f in ("assign_tc.cu", "tc_argmin.cuh", "fk_common.cuh"):
         with open(os.path.join(ROOT, "distance_argmin_flashassign_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
