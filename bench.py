@@ -229,6 +229,7 @@ def build_inputs(name: str, device, seed: int, rows: int = 0):
 # measured ones): dense fp16/bf16 tensor throughput and HBM3e bandwidth.
 SPEC_P16_TFLOPS = 2250.0
 TF32_PER_BF16 = 1.1 / 2.25  # nominal dense tf32 / bf16 rate
+SFU_EX2_PER_SM_CLK = 16     # ex2.approx per SM per clock (4 per sub-partition)
 SPEC_HBM_GBS = 8000.0
 
 
@@ -397,15 +398,22 @@ def measure_gauss(args, fk, dev, steps: int, warmup: int):
     peaks, peak_kind = load_peaks()
     flops = 2.0 * N * K * D
     tflops = flops / (ms * 1e-3) / 1e12
+    # one ex2 per (point, centroid) on the special-function units: 16 per SM
+    # per clock (4 per sub-partition), the bound this epilogue meets first
+    props = torch.cuda.get_device_properties(dev)
+    ex2_peak = props.multi_processor_count * SFU_EX2_PER_SM_CLK * SM_MAX_GHZ  # G ex2/s
+    ex2_rate = N * K / (ms * 1e-3) / 1e9
     return {"value": round(1e3 / ms, 3), "unit": "calls/s", "ms_per_step": round(ms, 5), "steps": steps,
             "config": {"workload": "gauss_f16", "N": N, "D": D, "K": K, "dtype": "f16", "beta": 2.0,
                        "weights": "uniform in [0.5, 1.5)",
                        "step": "fk_gauss_sum: Gauss-sum bias prep + tensor-core pass with a log-sum-exp epilogue"},
-            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (Gauss-sum epilogue)",
-                         "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tflops / peaks["bf16_tflops"], 4),
-                         "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
-                         "exp2_per_s": round(N * K / (ms * 1e-3), 1), "traffic": None},
+            "roofline": {"bound": "sfu", "kernel": "assign_tc_kernel (Gauss-sum epilogue)",
+                         "achieved": round(ex2_rate, 1), "peak": round(ex2_peak, 1), "unit": "G ex2/s",
+                         "frac": round(ex2_rate / ex2_peak, 4),
+                         "peak_kind": f"ex2: {props.multi_processor_count} SMs x {SFU_EX2_PER_SM_CLK} per clock x "
+                                      f"{SM_MAX_GHZ} GHz (derived from unit counts and clock)",
+                         "tensor_tflops": round(tflops, 2), "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
+                         "traffic": None},
             "clocks": clocks.summary(w0, w1)}
 
 
@@ -455,6 +463,49 @@ def measure_fused(args, fk, dev, reps: int):
             "clocks": clocks.summary(w0, w1)}
 
 
+def measure_top2(args, fk, dev, steps: int, warmup: int):
+    """The two nearest centroids of the embedding workload's points among its
+    K = 1,024 initial centroids (fk_assign_top2: the assignment stage twice,
+    the second pass leaving each point's nearest centroid out)."""
+    import torch
+    s, w = build_inputs("embed_f16", dev, 0)
+    X, C = w.X, w.C0.to(torch.float16)
+    N, D, K = s.N, s.D, s.K
+    l1 = torch.empty(N, dtype=torch.int32, device=dev)
+    l2 = torch.empty(N, dtype=torch.int32, device=dev)
+    for _ in range(warmup):
+        fk.fk_assign_top2(X, C, l1, l2)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(steps):
+        fk.fk_assign_top2(X, C, l1, l2)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    clocks.stop()
+    fk.fk_sync()
+    ms = e0.elapsed_time(e1) / steps
+    peaks, peak_kind = load_peaks()
+    flops = 2 * 2.0 * N * K * D  # two assignment passes
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"value": round(1e3 / ms, 3), "unit": "calls/s", "ms_per_step": round(ms, 5), "steps": steps,
+            "config": {"workload": "top2_f16", "N": N, "D": D, "K": K, "dtype": "f16",
+                       "step": "fk_assign_top2: bias prep, two tensor-core assignment passes (the second "
+                               "masking each point's nearest centroid), exact re-decision of near-ties after each"},
+            "roofline": {"bound": "tensor", "kernel": "assign_tc_kernel (argmin, then argmin with a mask)",
+                         "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tflops / peaks["bf16_tflops"], 4),
+                         "peak_kind": f"{peak_kind} bf16 burst (fp16 = bf16 dense rate)",
+                         "algorithmic_flops_per_call": flops, "traffic": None},
+            "clocks": clocks.summary(w0, w1)}
+
+
 def measure_seed(args, fk, dev, K: int):
     """k-means++ seeding of the embedding workload (N = 2^20, D = 128, fp16)
     with K centres: one kernel per centre (fp32-screened D2 update reading X
@@ -484,8 +535,8 @@ def measure_seed(args, fk, dev, K: int):
                          "algorithmic_bytes_per_round": bytes_per_round, "traffic": None}}
 
 
-OTHER_WORKLOADS = ("tiny_f32", "tiny_f32_fused", "batched_bf16", "zipf_bf16", "embed_f32", "gauss_f16", "seed_f16",
-                   "ooc_f16")
+OTHER_WORKLOADS = ("tiny_f32", "tiny_f32_fused", "batched_bf16", "zipf_bf16", "embed_f32", "gauss_f16", "top2_f16",
+                   "seed_f16", "ooc_f16")
 
 
 def bench_gpu(args):
@@ -533,6 +584,8 @@ def bench_gpu(args):
             others["tiny_f32_fused"] = measure_fused(args, fk, dev, max(3, min(args.steps, 40)))
         if "gauss_f16" in pick:
             others["gauss_f16"] = measure_gauss(args, fk, dev, max(3, min(args.steps, 50)), 3)
+        if "top2_f16" in pick:
+            others["top2_f16"] = measure_top2(args, fk, dev, max(3, min(args.steps, 50)), 3)
         if "seed_f16" in pick:
             others["seed_f16"] = measure_seed(args, fk, dev, 1024)
         torch.cuda.empty_cache()

@@ -245,7 +245,10 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
   const int NV = D / E;
   if (threadIdx.x == 0) sh_s = first ? 0 : weight_exponent(ctl, Lg);
   const int lane = threadIdx.x & 31, sub = lane % L, g = lane / L;
-  const int r0 = blockIdx.x * kSeedThreads + (threadIdx.x & ~31);
+  // serpentine order: odd rounds walk the row blocks backwards, so the first
+  // blocks to run read the rows the previous round read last (still in L2)
+  const int rb = (t & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  const int r0 = rb * kSeedThreads + (threadIdx.x & ~31);
   const int row_l = r0 + lane;  // the row this lane owns for the exact sum
   const uint4 *Xv = reinterpret_cast<const uint4 *>(X);
   double old = 0.0;
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
     return;
   }
   const long long b = block_sum(row_l < N ? weight_of(dn, sh_s) : 0, sm.ws);
-  if (threadIdx.x == 0) bsum[blockIdx.x] = b;
+  if (threadIdx.x == 0) bsum[rb] = b;
   draw_if_last<T>(sm, X, N, D, d2, u, t, bsum, sh_s, ctl, centers, crow);
 }
 
