@@ -25,7 +25,7 @@
 // Rows of a multiple of 16 bytes (16-byte aligned X) take one kernel per
 // round, seed_round_kernel: warp-cooperative 16-byte loads, the update of D2,
 // the blocks' weight sums and, in the last block to finish, the draw and the
-// next centre's row.  Round 1 (which also finds the largest D2, and so s)
+// next centre's row.  The first round (which also finds the largest D2, and so s)
 // adds seed_sample_kernel.  Other rows take seed_update_kernel +
 // seed_sample_kernel every round.
 #include "fk_internal.h"
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kSeedThreads) seed_round_kernel(const T *__res
 // first copies its 32 consecutive rows into shared memory with coalesced
 // 4-byte loads (rows padded by 4 bytes, so that the lanes' reads of one
 // dimension fall in different banks) where they fit; otherwise a thread reads
-// its row from global memory.  Round 1 also takes the largest D2.
+// its row from global memory.  The first round also takes the largest D2.
 template <typename T>
 __global__ void __launch_bounds__(kSeedThreads) seed_update_kernel(const T *__restrict__ X, int N, int D,
                                                                    const float *__restrict__ crow,

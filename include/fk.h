@@ -90,7 +90,7 @@ typedef int fk_status;
 enum {
   FK_OK = 0,
   FK_ERR_INVALID_ARG = -1, /* bad pointer, size or dtype                       */
-  FK_ERR_UNSUPPORTED = -2, /* valid request this build cannot run              */
+  FK_ERR_UNSUPPORTED = -2, /* valid request the library cannot serve          */
   FK_ERR_CUDA = -3,        /* a CUDA runtime call failed (no device, launch)   */
   FK_ERR_OOM = -4,         /* device or pinned allocation failed               */
   FK_ERR_TIMEOUT = -5,     /* a device-side wait exceeded its time limit       */
