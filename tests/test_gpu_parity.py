@@ -414,3 +414,37 @@ def test_launch_counter_counts_kernels():
     fk.fk_assign(X, X[:300].clone())
     fk.fk_sync()
     assert fk.fk_launch_count() - n0 == 3  # norms + tensor-core assign + near-tie re-decision
+
+
+TF32_SHAPES = [(1, 4, 1), (129, 1024, 129), (5000, 36, 4096), (300, 8, 2), (2048, 64, 257), (777, 4, 40)]
+
+
+@pytest.mark.parametrize("shape", TF32_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fp32_tensor_path_edges(shape):
+    """The fp32 tensor-core path (three tf32 passes) at its edges: one row, the
+    smallest and largest D it takes (4 and 1,024 = 32 k-blocks), ragged units
+    and tiles (129 rows and centroids), K = 1 to 4,096.  Forced onto that path;
+    labels must equal the oracle's."""
+    N, D, K = shape
+    X, C0 = mixture(N, D, K, "f32", seed=N * 7 + D + K)
+    try:
+        fk.fk_set_assign_path(1)
+        labels, mind = fk.fk_assign(X.to(DEV), C0.to(DEV), want_mindist=True)
+        fk.fk_sync()
+    finally:
+        fk.fk_set_assign_path(0)
+    check_labels(f64(X), f64(C0), labels, "f32", gpu_mindist=mind, exact=True,
+                 case=f"tf32 path {N}x{D}x{K}")
+
+
+def test_fp32_unaligned_rows_fall_back():
+    """X starting 4 bytes past a 16-byte boundary cannot feed the tensor maps:
+    the assignment runs on the CUDA-core kernel, with the same exact labels."""
+    X, C0 = mixture(3000, 64, 300, "f32", seed=77)
+    base = torch.empty(X.numel() + 1, device=DEV)
+    Xu = base[1:].view(X.shape)
+    Xu.copy_(X.to(DEV))
+    assert Xu.data_ptr() % 16 == 4
+    labels, mind = fk.fk_assign(Xu, C0.to(DEV), want_mindist=True)
+    fk.fk_sync()
+    check_labels(f64(X), f64(C0), labels, "f32", gpu_mindist=mind, exact=True, case="fp32 unaligned rows")
