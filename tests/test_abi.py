@@ -115,3 +115,28 @@ def test_debug_inject_arguments():
     assert fk.lib.fk_debug_inject(3, 0) == fk.FK_ERR_INVALID_ARG
     assert fk.lib.fk_debug_inject(1, -1) == fk.FK_ERR_INVALID_ARG
     assert fk.lib.fk_debug_inject(0, -1) == fk.FK_OK
+
+
+def test_new_entry_points_validate_on_the_host():
+    """Argument errors of the single-pass, top-2, Gauss and seeding calls are
+    reported before any device work (these run without a GPU)."""
+    p = ctypes.c_void_p(16)
+    q = ctypes.c_void_p(32)
+    lib = fk.lib
+    # single pass: iters < 1, a K x D too large for shared memory
+    assert lib.fk_lloyd_fused(p, 100, 8, 0, p, 4, p, None, None, 0, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_lloyd_fused(p, 100, 128, 0, p, 1024, p, None, None, 1, None) == fk.FK_ERR_UNSUPPORTED
+    assert "single-pass" in lib.fk_last_error_message().decode()
+    # top-2: aliased outputs, missing outputs
+    assert lib.fk_assign_top2(p, 100, 8, 0, p, 4, q, q, None, None, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_assign_top2(p, 100, 8, 0, p, 4, q, None, None, None, None) == fk.FK_ERR_INVALID_ARG
+    # Gauss sums: beta, signed weights without weights, no output
+    f = ctypes.c_float
+    assert lib.fk_gauss_sum(p, 100, 8, 0, p, 4, None, 0, f(0.0), q, None, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_gauss_sum(p, 100, 8, 0, p, 4, None, 1, f(1.0), q, None, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_gauss_sum(p, 100, 8, 0, p, 4, None, 0, f(1.0), None, None, None) == fk.FK_ERR_INVALID_ARG
+    # seeding: a uniform outside [0, 1), N = 0
+    import numpy as np
+    u = np.array([0.5, 1.0], dtype=np.float64)
+    assert lib.fk_seed_kmeanspp(p, 100, 8, 0, 2, ctypes.c_void_p(u.ctypes.data), q, None) == fk.FK_ERR_INVALID_ARG
+    assert lib.fk_seed_kmeanspp(p, 0, 8, 0, 2, ctypes.c_void_p(u.ctypes.data), q, None) == fk.FK_ERR_INVALID_ARG
