@@ -767,7 +767,10 @@ uint64_t fk_launch_count(void) { return g_launches.load(); }
 
 int fk_assign_path(int64_t N, int D, fk_dtype dt, int K, int B) {
   if (!valid_dtype(dt) || B < 1 || N < 0 || D < 1 || D > 1024 || K < 1) return FK_ERR_INVALID_ARG;
-  return choose_path((DType)dt, D);
+  const int path = choose_path((DType)dt, D);
+  // the fp32 tensor path takes one problem at a time; a batch runs on CUDA cores
+  if (path == 1 && (DType)dt == kF32 && B > 1) return g_assign_path.load() == 1 ? FK_ERR_UNSUPPORTED : 2;
+  return path;
 }
 
 fk_status fk_set_assign_path(int path) {

@@ -23,8 +23,10 @@
  *   dtype      FK_F32, FK_F16 or FK_BF16 tags the element type of X (and of C
  *              where C is given in the input type).  Arithmetic accumulates in
  *              fp32.  fp16/bf16 assignment runs on tcgen05 tensor cores when
- *              D is a multiple of 8 and 8 <= D <= 256; every other case runs on
- *              a CUDA-core kernel (fp32 always does).
+ *              D is a multiple of 8 and 8 <= D <= 256; fp32 assignment of one
+ *              problem with D a multiple of 4 (16-byte aligned X and C) runs on
+ *              them as three tf32 passes on split hi/lo operands; every other
+ *              case runs on a CUDA-core kernel.
  *   Distances  label[i] = argmin_k |x_i - c_k|^2 with ties to the LOWEST k
  *              (the pages are silent on ties).  mindist[i] = that squared
  *              distance, clamped at 0.  The tensor path ranks by
@@ -323,8 +325,8 @@ FK_API fk_status fk_lloyd_ooc(const void *X_host, int64_t N, int D, fk_dtype dt,
  *   beta     > 0
  *   G        device, N fp32 (out) or NULL; may underflow or overflow in fp32
  *   logG     device, N fp32 (out) or NULL: ln G (NaN where G <= 0)
- *   fp16/bf16 with D % 8 == 0, D <= 256 run on tcgen05; other inputs on a
- *   CUDA-core kernel.  Asynchronous on `stream`.
+ *   fp16/bf16 with D % 8 == 0, D <= 256 run on tcgen05; other inputs (fp32
+ *   included) on a CUDA-core kernel.  Asynchronous on `stream`.
  * ------------------------------------------------------------------------ */
 FK_API fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, const void *C, int K, const float *w,
                               int w_signed, float beta, float *G, float *logG, fk_stream_t stream);
@@ -370,8 +372,10 @@ FK_API const char *fk_last_error_message(void);
 FK_API uint64_t fk_launch_count(void);
 
 /* Which assignment kernel fk_assign would run for this request:
- * 1 = tcgen05 tensor-core kernel, 2 = CUDA-core kernel, or a negative status
- * for an invalid request.  Host-only: queries no device. */
+ * 1 = tcgen05 tensor-core kernel (fp32: three tf32 passes), 2 = CUDA-core
+ * kernel, or a negative status for an invalid request (or, under a forced
+ * tensor path, one it cannot serve).  Host-only: queries no device; a tensor
+ * answer still needs 16-byte aligned X and C at the call. */
 FK_API int fk_assign_path(int64_t N, int D, fk_dtype dt, int K, int B);
 
 /* Force the assignment kernel: 0 = automatic (default), 1 = tensor-core

@@ -44,6 +44,7 @@ def test_assign_path_choice():
     assert fk.fk_assign_path(1000, 8, torch.float16, 3) == 1
     assert fk.fk_assign_path(1000, 32, torch.float32, 128) == 1   # fp32: three tf32 passes on tensor cores
     assert fk.fk_assign_path(1000, 30, torch.float32, 128) == 2   # fp32 rows not whole 16-byte groups
+    assert fk.fk_assign_path(1000, 32, torch.float32, 128, B=3) == 2  # a batch of fp32 problems
     assert fk.fk_assign_path(1000, 100, torch.float16, 8) == 2    # D not a multiple of 8
     assert fk.fk_assign_path(1000, 256, torch.float16, 8) == 1    # up to 256 dimensions on tensor cores
     assert fk.fk_assign_path(1000, 264, torch.float16, 8) == 2    # D above 256
