@@ -223,9 +223,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full(s), 1);   // the leader's expect_tx; bytes from both CTAs
       mbar_init(empty(s), 1);  // the epilogue, once the tile using the slot is complete
     }
+    // With one tile per unit and |x|^2 prepared, nothing but the MMAs reads an
+    // X buffer: the MMA thread's commit frees it as soon as they complete.
+    // Otherwise this CTA's epilogue warps of the unit free it after the unit.
+    const bool x_by_mma = p.ntiles == 1 && p.xnorm != nullptr;
     for (int x = 0; x < XBUF; ++x) {
       mbar_init(xfull(x), 1);
-      mbar_init(xempty(x), p.ntiles == 1 ? kEpiWarps / 2 : kEpiWarps);  // this CTA's warps of the unit, after it
+      mbar_init(xempty(x), x_by_mma ? 1 : p.ntiles == 1 ? kEpiWarps / 2 : kEpiWarps);
       mbar_init(xready(x), 1);  // one leader warp of the unit (read in the peer, one tile per unit)
     }
     // With one tile per unit each unit is read by one warp of each lane
@@ -357,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit_pair(accfull(a), kBothCtas);
         }
         if (!ok) break;
+        if (p.ntiles == 1 && p.xnorm) tc_commit_pair(xempty(xb), kBothCtas);  // the unit's MMAs have read X
         if (++xb == XBUF) { xb = 0; xph ^= 1u; }
       }
       // Every MMA this thread issued completes before TMEM is released (all
@@ -500,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           list_near_tie(p.ties, row < p.N, bs.score, s2, bs.s3, xn, o_, bs.base2);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(xempty(xb));
+        if (lane == 0 && !p.xnorm) mbar_arrive(xempty(xb));  // (with |x|^2 prepared the MMA commit frees it)
       }
     } else {
       uint32_t xb = 0, xc = 0;
