@@ -15,8 +15,9 @@
 // Per iteration, per CTA:
 //   1. the centroids C_t, rounded to the input type, into shared memory;
 //   2. passes of 512 / S rows: S threads share a row (S grows for small N
-//      so that every SM gets rows), each taking every S-th tile of 32
-//      centroids, with the fp32 direct difference (as the CUDA-core
+//      so that every SM gets rows), thread s taking the centroids
+//      k0 + t S + s of each block of 32 S, with the fp32 direct difference
+//      (as the CUDA-core
 //      assignment kernel), keeping the best and second-best distance; a row
 //      whose two lie within the fp32 rounding bound of each other is
 //      re-decided exactly by its warp, over every centroid, with the fp64
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(kFzThreads) lloyd_fused_kernel(FzArgs a) {
     __syncthreads();
     for (int p = 0; p < npass; ++p) {
       // S threads share a row (adjacent lanes); thread s of a row takes the
-      // 32-centroid tiles s, s + S, s + 2S, ...
+      // centroids k0 + t S + s (t < 32) of each block of 32 S centroids, so
+      // the S threads read S consecutive centroid rows at once
       const int r0 = (p * G + blockIdx.x) * P;
       const int prow = tid / S, sub = tid % S;
       const int row = r0 + prow;
