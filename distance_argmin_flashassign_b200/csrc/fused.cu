@@ -17,8 +17,8 @@
 //   2. passes of 512 / S rows: S threads share a row (S grows for small N
 //      so that every SM gets rows), thread s taking the centroids
 //      k0 + t S + s of each block of 32 S, with the fp32 direct difference
-//      (as the CUDA-core
-//      assignment kernel), keeping the best and second-best distance; a row
+//      (as the CUDA-core assignment kernel), keeping the best and
+//      second-best distance; a row
 //      whose two lie within the fp32 rounding bound of each other is
 //      re-decided exactly by its warp, over every centroid, with the fp64
 //      direct difference and the lowest index on ties -- so every label is
