@@ -354,9 +354,22 @@ size_t tf32_workspace_bytes(int64_t N, int D, int K) {
   return 2 * al((size_t)N * D * 4) + al((size_t)N * 4) + 2 * al((size_t)K * D * 4);
 }
 
+cudaError_t launch_tf32_split_points(const float *X, int N, int D, void *ws, cudaStream_t s) {
+  auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+  char *w = (char *)ws;
+  float *xh = (float *)w; w += al((size_t)N * D * 4);
+  float *xl = (float *)w; w += al((size_t)N * D * 4);
+  float *xn = (float *)w;
+  long long g = ((long long)N * 32 + 255) / 256;
+  g = g < 4096 ? (g > 0 ? g : 1) : 4096;
+  tf32_split_kernel<<<(int)g, 256, 0, s>>>(X, N, D, xh, xl, xn);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_assign_tf32(const float *X, const float *C, const float *bias, int N, int D, int K, int Kpad,
                                int32_t *labels, float *mindist, NearTies ties, void *ws, DevCtl ctl, int num_sms,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool x_split) {
   if (!tf32_shape_ok(D) || (uintptr_t)bias % 16 != 0) return cudaErrorNotSupported;
   if (Kpad < (K + kF32TileN - 1) / kF32TileN * kF32TileN) return cudaErrorInvalidValue;
   auto al = [](size_t v) { return (v + 255) / 256 * 256; };
@@ -370,9 +383,12 @@ cudaError_t launch_assign_tf32(const float *X, const float *C, const float *bias
     long long g = (rows * 32 + 255) / 256;
     return (int)(g < 4096 ? (g > 0 ? g : 1) : 4096);
   };
-  tf32_split_kernel<<<grid_for(N), 256, 0, s>>>(X, N, D, xh, xl, xn);
+  if (!x_split) {  // (a Lloyd run splits X once: the points do not change)
+    tf32_split_kernel<<<grid_for(N), 256, 0, s>>>(X, N, D, xh, xl, xn);
+    count_launches(1);
+  }
   tf32_split_kernel<<<grid_for(K), 256, 0, s>>>(C, K, D, ch, cl, nullptr);
-  count_launches(2);
+  count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap xhm, xlm, chm, clm, bm;

@@ -218,7 +218,7 @@ static int choose_path(DType dt, int D) {
 // kernel then computes it from its X tiles.
 static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, int D, const void *C, int K,
                             const float *cn, float *cn_ws, void *ties_ws, const float *xnorm, int32_t *labels,
-                            float *mindist, cudaStream_t s, const int32_t *excl = nullptr) {
+                            float *mindist, cudaStream_t s, const int32_t *excl = nullptr, bool x_split = false) {
   NearTies ties;
   fk_status st = near_ties(d, s, ties_ws, (int64_t)B * N, D, &ties);
   if (st != FK_OK) return st;
@@ -240,7 +240,7 @@ static fk_status run_assign(DevState &d, DType dt, const void *X, int B, int N, 
       NearTies tt = ties;
       tt.tau = near_tie_tau_tf32(D);
       cudaError_t e = launch_assign_tf32((const float *)X, (const float *)C, cn, N, D, K, Kpad, labels, mindist, tt,
-                                         aux, ctl_of(d), d.sms, s);
+                                         aux, ctl_of(d), d.sms, s, x_split);
       if (e == cudaSuccess) {
         done = true;
       } else {
@@ -501,6 +501,15 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
   a.C = C;
   a.counts = counts;
   a.mode = kMean;
+  // fp32 on the tensor path: X's tf32 split is made once for all iterations
+  bool x_split = false;
+  if (t == kF32 && B == 1 && choose_path(t, D) == 1 && tc_aligned(X, C) && (uintptr_t)cn % 16 == 0) {
+    void *aux = nullptr;
+    if ((st = aux_scratch(*d, s, tf32_workspace_bytes(N, D, K), &aux)) != FK_OK) return st;
+    cudaError_t e = launch_tf32_split_points((const float *)X, (int)N, D, aux, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tf32 split kernel");
+    x_split = true;
+  }
   for (int it = 0; it < iters; ++it) {
     {  // the centroids as the assignment reads them (fp16/bf16: rounded) and their bias
       cudaError_t e = t != kF32 ? launch_round_bias(t, C, B, K, Kpad, D, Cdt, cn, s)
@@ -508,7 +517,7 @@ fk_status fk_lloyd_batched(const void *X, int B, int64_t N, int D, fk_dtype dt, 
       if (e != cudaSuccess) return cuda_fail(e, "centroid prep kernel");
     }
     st = run_assign(*d, t, X, B, (int)N, D, Cdt, K, cn, nullptr, tl, xn, labels, it == iters - 1 ? mindist : nullptr,
-                    s);
+                    s, nullptr, x_split);
     if (st != FK_OK) return st;
     cudaError_t e = launch_update(a, ws, upd, ctl_of(*d), d->sms, s);
     if (e != cudaSuccess) return cuda_fail(e, "update kernels");

@@ -30,9 +30,13 @@ bool tf32_shape_ok(int D);
 size_t tf32_workspace_bytes(int64_t N, int D, int K);
 // One problem; ws of tf32_workspace_bytes(N, D, K).  cudaErrorNotSupported when
 // the shape or the tensor maps do not fit.
+// x_split: the workspace already holds X's split and |x|^2 (from
+// launch_tf32_split_points on the same X), so only C is split.
 cudaError_t launch_assign_tf32(const float *X, const float *C, const float *bias, int N, int D, int K, int Kpad,
                                int32_t *labels, float *mindist, NearTies ties, void *ws, DevCtl ctl, int num_sms,
-                               cudaStream_t s);
+                               cudaStream_t s, bool x_split = false);
+// The split of X (hi, lo) and |x|^2 into the workspace of launch_assign_tf32.
+cudaError_t launch_tf32_split_points(const float *X, int N, int D, void *ws, cudaStream_t s);
 
 // ---- fused.cu: single-pass Lloyd iterations (centroids in shared memory) ---
 // True when K x D fits the single-pass kernel's shared memory.
