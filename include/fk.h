@@ -339,14 +339,16 @@ FK_API fk_status fk_gauss_sum(const void *X, int64_t N, int D, fk_dtype dt, cons
  *   probability proportional to D2(x) = min over the centres so far of
  *   |x - c|^2, with these reproducible rules: D2 is sum_j (x_j - c_j)^2 in
  *   fp64, j ascending, each operation rounded; the weights are the integers
- *   floor(D2 2^s), s the largest exponent with N max D2 2^s < 2^61 for the
- *   D2 after the first centre; r = floor(u[t] T) for the weights' total T
+ *   floor(D2 2^s) with s = 61 - e - L, where the largest D2 after the first
+ *   centre is m 2^e (m in [1/2, 1)) and 2^L >= N, so that the total stays
+ *   below 2^61; r = floor(u[t] T) for the weights' total T
  *   (T - 1 if that rounds up to T), and the centre is the first point whose
  *   running weight exceeds r; with T = 0 it is point floor(u[t] N).
  *   X        device, N x D, dtype dt, N >= 1
  *   u        host, K doubles in [0, 1): the draws (the caller's generator)
  *   centers  device, K int32 (out): row indices of the chosen centres
- *   Scratch 8 N bytes and a little more.  Two kernels per centre.
+ *   Scratch 8 N bytes and a little more.  One kernel per centre when a row
+ *   is a whole number of 16 bytes (16-byte aligned X), two otherwise.
  *   Synchronises `stream`.
  * ------------------------------------------------------------------------ */
 FK_API fk_status fk_seed_kmeanspp(const void *X, int64_t N, int D, fk_dtype dt, int K, const double *u,
